@@ -1,0 +1,318 @@
+"""Benchmark of the SageAttention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sage|reference]
+                    [--workload NAME] [--extra-workloads a,b] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the whole path over one batch of synthetic input:
+sage_quant_qkv (smooth K / smooth Q + delta_S, INT8 Q/K, FP8 V) followed by
+the fused INT8/FP8 attention kernel.  The metric is attention TOPS
+(4 N^2 d per head, halved when causal).  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the plain scalar reference of the
+method) on a bounded sample of the same workload on the host cores.
+Multi-GPU (torchrun): every rank runs the same per-GPU workload (weak
+scaling, no collective on the data path); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+_ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, _ROOT)
+
+from quantized_attention_block_b200 import workloads as W  # noqa: E402
+
+INT8_FP8_PER_BF16 = 2.0  # nominal dense ratio 4.5 / 2.25 PFLOP/s
+
+
+def _peaks():
+    path = os.path.join(_ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+def _barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: int, e2e: bool):
+    from quantized_attention_block_b200 import sage
+
+    q, k, v = W.make_qkv(w, seed=w.seed + rank)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    p = sage.make_params(qd, kd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                         smooth_q=w.smooth_q, bq=w.bq, bk=w.bk)
+    wsp = sage.alloc_workspace(p)
+    o = torch.empty_like(qd)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        view = sage.sage_quant_qkv(qd, kd, vd, p, wsp, stream)
+        if ev is not None:
+            ev[0].record(stream)
+        sage.sage_attn_fwd_quantized(view, o, p, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(max(3, warmup)):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = 4 + (1 if w.smooth_q else 0)
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        _barrier(ws)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(steps):
+            step(attn_ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        _barrier(ws)
+    ms_total = t0.elapsed_time(t1)
+    ms_attn = sum(a.elapsed_time(b) for a, b in attn_ev) / steps
+    assert sage.sage_last_device_error() == 0
+    ms_step = _max_over_ranks(ms_total / steps, ws)
+    ms_attn = _max_over_ranks(ms_attn, ws)
+    res = {"ms_step": ms_step, "ms_attn": ms_attn, "ms_quant": ms_step - ms_attn, "clocks": clk.summary(),
+           "gpu_launches": launches_per_step * steps}
+
+    if e2e:
+        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            sage.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                               smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, out=o, workspace=wsp, stream=stream)
+            oh.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e_steps = max(3, min(steps, 10))
+        _barrier(ws)
+        t0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = _max_over_ranks(t0.elapsed_time(t1) / e_steps, ws)
+        res["e2e"] = {"ms_step": ms_e2e, "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                      "d2h_bytes_per_step": o.numel() * o.element_size(), "steps": e_steps}
+    del wsp, qd, kd, vd, o
+    torch.cuda.empty_cache()
+    return res
+
+
+def oracle_sample(w: W.Workload, heads: int, tiles: int, threads: int):
+    """Time the CPU oracle on a bounded sample: quantise `heads` (b, h) pairs
+    and run the attention of the last `tiles` Q tiles of each (the longest rows
+    when causal).  Returns (seconds, attention ops of the sample, description)."""
+    import numpy as np
+
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+
+    G = w.Hq // w.Hkv
+    sw = w.with_(B=1, Hq=heads * G if w.Hq != w.Hkv else heads, Hkv=heads if w.Hq != w.Hkv else heads)
+    q, k, v = W.make_qkv(sw)
+    n_t = -(-w.N // 128)
+    jobs = [(0, h, t * 128, min((t + 1) * 128, w.N)) for h in range(sw.Hq) for t in range(n_t - tiles, n_t)]
+    ops = 0.0
+    for _, _, r0, r1 in jobs:
+        for r in range(r0, r1):
+            keys = (r + 1) if w.causal else w.N
+            ops += 4.0 * keys * w.d
+    t_start = time.perf_counter()
+    quant = oracle.quantize_sage(q, k, v, bq=w.bq, bk=w.bk, smooth_k=w.smooth_k, smooth_q=w.smooth_q,
+                                 threads=threads)
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda j: oracle.attention_sage_head(quant, j[0], j[1], j[2], j[3], bq=w.bq, bk=w.bk,
+                                                        causal=w.causal, sm_scale=w.sm_scale), jobs))
+    secs = time.perf_counter() - t_start
+    desc = (f"{sw.Hq} heads of {w.name} (B=1, N={w.N}): full oracle quantisation of those heads + "
+            f"attention of the last {tiles} Q tiles of each ({len(jobs)} tiles), {threads} threads")
+    return secs, ops, desc
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sage", "reference"], default="sage")
+    ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--extra-workloads", default="video,gqa")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    ws, rank, local = _dist()
+    w = W.get(args.workload)
+    metric = "quantized attn fwd TOPS on 1 B200 (N=4K-32K, d=64/128); % of tensor peak"
+    threads = os.cpu_count() or 1
+    config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+              "causal": w.causal, "smooth_q": w.smooth_q, "bq": w.bq, "bk": w.bk,
+              "input_dtype": str(w.dtype).replace("torch.", ""), "parallelism": f"replicas x{ws} (weak)",
+              "l2": "inputs larger than L2 (Q/K/V bf16 and their quantised copies each exceed 126 MB)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        heads, tiles = (4, 2) if w.N >= 8192 else (8, 4)
+        vals = []
+        desc = ""
+        if args.warmup > 0:
+            oracle_sample(w, 1, 1, threads)
+        for _ in range(args.steps):
+            secs, ops, desc = oracle_sample(w, heads, tiles, threads)
+            vals.append(ops / secs / 1e12)
+        val = statistics.median(vals)
+        print(json.dumps({
+            "impl": "reference", "metric": metric, "value": val, "unit": "TOPS", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (int8/e4m3 codes, fp32 state)", "data": "synthetic",
+            "config": config,
+            "cpu_baseline": {"value": val, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    if ws > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                             timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+
+    peaks, peak_kind = _peaks()
+    peak_tops = peaks["bf16_tflops_sustained"] * INT8_FP8_PER_BF16
+    res = run_sage(w, args.steps, args.warmup, ws, rank, local, not args.no_e2e)
+    ops = w.ops()
+    value = ws * ops / (res["ms_step"] * 1e-3) / 1e12
+    attn_tops = ops / (res["ms_attn"] * 1e-3) / 1e12
+    extra = {}
+    for name in [x for x in args.extra_workloads.split(",") if x and x != "none"]:
+        we = W.get(name)
+        r = run_sage(we, max(3, args.steps // 4), 3, ws, rank, local, False)
+        extra[we.name] = {"step_tops": we.ops() / (r["ms_step"] * 1e-3) / 1e12,
+                          "attn_kernel_tops": we.ops() / (r["ms_attn"] * 1e-3) / 1e12,
+                          "ms_step": r["ms_step"], "ms_attn": r["ms_attn"],
+                          "attn_frac_of_peak": we.ops() / (r["ms_attn"] * 1e-3) / 1e12 / peak_tops}
+    line = {
+        "metric": metric, "value": value, "unit": "TOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": res["ms_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8+e4m3 (fp32 accumulate)",
+        "data": "synthetic (seeded, recipe of the workload)", "config": config,
+        "kernel_only_tops": attn_tops,
+        "per_kernel_ms": {"quant_total": res["ms_quant"], "attn_i8f8": res["ms_attn"]},
+        "roofline": {"bound": "tensor", "kernel": "attn_i8f8_kernel", "achieved": attn_tops,
+                     "peak": peak_tops, "unit": "TFLOP/s", "frac": attn_tops / peak_tops,
+                     "peak_source": f"{peak_kind}: bf16 sustained {peaks['bf16_tflops_sustained']} x "
+                                    f"{INT8_FP8_PER_BF16} (nominal int8/fp8 : bf16)",
+                     "traffic": None},
+        "clocks": res["clocks"], "gpu_launches": res["gpu_launches"], "workloads": extra,
+    }
+    if "e2e" in res:
+        e = res["e2e"]
+        line["e2e"] = {"value": ws * ops / (e["ms_step"] * 1e-3) / 1e12, "unit": "TOPS",
+                       "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
+                       "ms_step": e["ms_step"]}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        secs, ops_s, desc = oracle_sample(w, 8, 4, threads)
+        line["cpu_baseline"] = {"value": ops_s / secs / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                                "sample": desc, "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line))
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,160 @@
+/*
+ * sage.h -- C ABI of libsage, a B200 (sm_100a) implementation of the
+ * SageAttention quantized attention forward pass.
+ *
+ * Method (cited by page title and section):
+ *   - "SageAttention2: Efficient Attention with Thorough Outlier Smoothing and
+ *     Per-thread INT4 Quantization" reading note
+ *     (zhaifeiyue.github.io/papers/2411.10958/detail), Algorithm 1: smooth K,
+ *     smooth Q with the delta_S GEMV compensation, per-block INT8 Q/K,
+ *     per-channel FP8 V, online softmax, P~ * 448 -> E4M3, FP8 PV with
+ *     two-level FP32 accumulation, final O / l / 448 * delta_V.
+ *   - "FlashAttention vs SageAttention" source note (kenforever1.github.io),
+ *     sections "执行流水线" and "后端矩阵": the API takes Q/K/V, layout,
+ *     is_causal, sm_scale; fp16/bf16 inputs only; head_dim 64/128 (larger is
+ *     rejected); GQA needs Hq % Hkv == 0; smooth_k subtracts the token mean
+ *     of K, broadcast to the Q heads of a KV group.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are HND: [B, H, N, d], contiguous, d fastest.
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *     stated otherwise; the library never allocates device memory.  Scratch
+ *     lives in a caller-provided workspace of sage_workspace_bytes() bytes.
+ *   - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; argument errors are returned synchronously and
+ *     nothing is enqueued.  Device-side failures (a bounded wait inside a
+ *     kernel that gave up) are reported by sage_last_device_error().
+ *   - Only sm_100 devices are accepted (SAGE_ERR_UNSUPPORTED_ARCH otherwise).
+ */
+#ifndef SAGE_H
+#define SAGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAGE_API __attribute__((visibility("default")))
+#else
+#define SAGE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARG = 1,          /* null pointer, bad sizes, Hq % Hkv != 0, N < 1 ... */
+    SAGE_ERR_UNSUPPORTED_HEADDIM = 2,  /* d not in {64, 128} */
+    SAGE_ERR_UNSUPPORTED_DTYPE = 3,    /* dtype not bf16/fp16 */
+    SAGE_ERR_UNSUPPORTED_ARCH = 4,     /* current device is not sm_100 */
+    SAGE_ERR_WORKSPACE_TOO_SMALL = 5,
+    SAGE_ERR_CUDA = 6,                 /* a CUDA runtime/driver call failed */
+    SAGE_ERR_TIMEOUT = 7,              /* a bounded in-kernel wait gave up */
+    SAGE_ERR_MISALIGNED = 8            /* a pointer is not 16-byte aligned */
+} sage_status;
+
+typedef enum { SAGE_BF16 = 0, SAGE_FP16 = 1 } sage_dtype;
+
+/* Problem description shared by all entry points. */
+typedef struct {
+    int32_t B, Hq, Hkv, N, d;  /* batch, query heads, key/value heads, tokens, head_dim */
+    int32_t dtype;             /* sage_dtype of Q, K, V and O */
+    int32_t causal;            /* 1: key j > query i is masked (top-left aligned) */
+    float   sm_scale;          /* softmax scale; <= 0 selects 1/sqrt(d) */
+    int32_t smooth_k;          /* 1: subtract the per-(b, kv-head, channel) token mean of K */
+    int32_t smooth_q;          /* 1: subtract each Q block's mean and add delta_S back */
+    int32_t bq;                /* Q quantisation block in rows: 64 or 128 */
+    int32_t bk;                /* K quantisation block in rows: 64 or 128 */
+} sage_params;
+
+/*
+ * Device views of the quantised tensors produced by sage_quant_qkv (all
+ * pointers point into the caller's workspace).  Np = N rounded up to 128
+ * (the attention kernel's tile); padded rows/columns hold zeros.
+ * Tm = ceil(N / bq), Tn = ceil(N / bk).
+ */
+typedef struct {
+    int8_t  *q8;    /* [B, Hq,  Np, d]  INT8 codes of (Q - qbar) or Q            */
+    int8_t  *k8;    /* [B, Hkv, Np, d]  INT8 codes of gamma(K) = K - km          */
+    uint8_t *v8t;   /* [B, Hkv, d, Np]  E4M3 codes of V / s_v, transposed        */
+    float   *s_q;   /* [B, Hq,  Tm]     delta_Q: amax/127 per Q block            */
+    float   *s_k;   /* [B, Hkv, Tn]     delta_K: amax/127 per K block            */
+    float   *s_v;   /* [B, Hkv, d]      delta_V: amax/448 per channel            */
+    float   *km;    /* [B, Hkv, d]      mean(K) over tokens (zeros if !smooth_k) */
+    float   *qbar;  /* [B, Hq,  Tm, d]  Q block means (NULL unless smooth_q)     */
+    float   *dS;    /* [B, Hq,  Tm, Np] delta_S = qbar . gamma(K)^T (or NULL)     */
+    int64_t  Np;
+} sage_quant_view;
+
+/* Bytes of workspace the entry points below need for `p` (0 if p is invalid). */
+SAGE_API size_t sage_workspace_bytes(const sage_params *p);
+
+/*
+ * Preprocessing of SageAttention2 Algorithm 1 ("Preprocessing" and the
+ * per-block psi_Q / psi_K quantisers; Figure 3 stages 1-3):
+ *   km      = mean_n K[b,g,n,:]              (fp64 sum, one rounding to fp32)
+ *   gamma K = K - km                         (fp32)
+ *   qbar_i  = mean of Q block i (smooth_q)   (fp64 sum over valid rows)
+ *   s_q/s_k = amax_block |x| / 127,  code = clamp(rint(x / s), -127, 127)
+ *   s_v[c]  = amax_n |V[n,c]| / 448, v8t   = E4M3_rn_satfinite(V / s_v)
+ *   dS[i,j] = qbar_i . gamma(K_j)            (smooth_q only; fp32 accumulation)
+ * q, k, v: device [B,H,N,d] in p->dtype.  Fills *view (host struct) with
+ * pointers into `workspace`.  Quantised tensors and scales are bit-exact with
+ * the plain definitions above.
+ */
+SAGE_API sage_status sage_quant_qkv(const void *q, const void *k, const void *v, const sage_params *p,
+                           void *workspace, size_t workspace_bytes,
+                           sage_quant_view *view, void *stream);
+
+/*
+ * The fused attention kernel of SageAttention2 Algorithm 1 (inner loop) on
+ * already-quantised tensors: per 128-row Q tile and 128-key K tile,
+ *   S   = (Q^ K^T)_int32 * s_q * s_k (+ dS) * sm_scale      (tcgen05 kind::i8)
+ *   m   = max(m, rowmax S); P~ = exp(S - m); l = e^(m_old-m) l + rowsum P~
+ *   O_t = E4M3(448 P~) @ V^                                (tcgen05 kind::f8f6f4,
+ *                                                            fresh TMEM tile)
+ *   O   = e^(m_old - m) O + O_t                             (FP32, CUDA cores)
+ * and finally O / l / 448 * s_v written to `o` [B,Hq,N,d] in p->dtype.
+ * `view` must come from sage_quant_qkv with the same p.
+ */
+SAGE_API sage_status sage_attn_fwd_quantized(const sage_quant_view *view, void *o, const sage_params *p,
+                                    void *stream);
+
+/* sage_quant_qkv followed by sage_attn_fwd_quantized (the whole forward). */
+SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, void *o, const sage_params *p,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Bit-exactness probe of the INT8 tensor-core path: the raw INT32 tile
+ * (Q^ K^T) for rows [128*qtile, +128) of head (b, h) and keys [128*ktile, +128),
+ * computed with the same TMA staging, shared-memory descriptors and
+ * tcgen05.mma kind::i8 instruction as the attention kernel, written
+ * row-major to out_128x128 (device, 128*128 int32).
+ */
+SAGE_API sage_status sage_debug_qk_int32(const sage_quant_view *view, const sage_params *p,
+                                int32_t b, int32_t h, int32_t qtile, int32_t ktile,
+                                int32_t *out_128x128, void *stream);
+
+/*
+ * Returns the first device-side error recorded since the last call
+ * (SAGE_OK or SAGE_ERR_TIMEOUT) and clears it.  Synchronises `stream`.
+ */
+SAGE_API sage_status sage_last_device_error(void *stream);
+
+/*
+ * Failure-detection check: launches one CTA that waits on an mbarrier nobody
+ * arrives at, bounded by `timeout_us`.  The wait gives up, records
+ * SAGE_ERR_TIMEOUT and the kernel returns normally (the context stays
+ * usable).  Returns the status sage_last_device_error() then reports.
+ */
+SAGE_API sage_status sage_debug_bounded_wait(uint32_t timeout_us, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+SAGE_API const char *sage_status_string(sage_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGE_H */

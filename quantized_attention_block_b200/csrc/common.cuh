@@ -1,0 +1,59 @@
+// common.cuh -- argument blocks shared by the host entry points (api.cu) and
+// the kernels (quant.cu, attn_i8f8.cu).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace sage {
+
+constexpr int kTile = 128;  // attention tile: 128 Q rows x 128 keys
+
+struct QuantArgs {
+  const void* q;  // [B,Hq,N,D] bf16/fp16
+  const void* k;  // [B,Hkv,N,D]
+  const void* v;  // [B,Hkv,N,D]
+  int B, Hq, Hkv, N, D;
+  int64_t Np;
+  int Tm, Tn, bq, bk;
+  int smooth_k, smooth_q;
+  // outputs / scratch (workspace)
+  int8_t* q8;
+  int8_t* k8;
+  uint8_t* v8t;
+  float* s_q;
+  float* s_k;
+  float* s_v;
+  float* km;
+  float* qbar;
+  float* dS;
+  double* ksum;     // [B,Hkv,D] fp64 column sums of K
+  unsigned* vamax;  // [B,Hkv,D] bit pattern of max |V| (non-negative floats order as uints)
+};
+
+struct AttnArgs {
+  int B, Hq, Hkv, N, D;
+  int64_t Np;
+  int Tm, Tn, bq, bk;
+  int causal;
+  int n_qtiles;
+  float scale_log2;  // sm_scale * log2(e)
+  const float* s_q;
+  const float* s_k;
+  const float* s_v;
+  const float* dS;  // nullptr when smooth_q is off
+  void* o;          // [B,Hq,N,D] bf16/fp16
+  int out_fp16;
+  // probe mode (sage_debug_qk_int32)
+  int probe_b, probe_h, probe_qtile, probe_ktile;
+  int32_t* probe_out;
+};
+
+// launchers (defined in the .cu files)
+cudaError_t launch_quant(const QuantArgs& a, int is_fp16, cudaStream_t st);
+cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, cudaStream_t st);
+cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, cudaStream_t st);
+cudaError_t launch_bounded_wait_probe(cudaStream_t st);
+
+}  // namespace sage

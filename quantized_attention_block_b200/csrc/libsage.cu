@@ -1,0 +1,6 @@
+// libsage.cu -- single translation unit for the library (the device-side
+// error word and wait limit are shared by all kernels without relocatable
+// device code).
+#include "quant.cu"
+#include "attn_i8f8.cu"
+#include "api.cu"

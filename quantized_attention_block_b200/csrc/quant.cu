@@ -1,0 +1,403 @@
+// quant.cu -- SageAttention preprocessing on sm_100a (HBM-bound kernels).
+//
+// Follows the "Preprocessing" part of Algorithm 1 in the SageAttention2 note
+// (zhaifeiyue.github.io/papers/2411.10958/detail) and Figure 3 stages 1-3:
+//   smooth K:  km = mean_n K,  gamma(K) = K - km               (exact shift)
+//   smooth Q:  qbar_i = mean of Q block i,  Q_i - qbar_i
+//   psi_Q/psi_K: per-block INT8, scale = amax / 127, code = rint(x / scale)
+//   psi_V:     per-channel FP8 E4M3, scale = amax / 448
+//   GEMV:      delta_S[i, j] = qbar_i . gamma(K_j)
+// Bit-exactness with the plain definitions: column sums are accumulated in
+// fp64 (the partial sums of bf16/fp16 inputs are exact, so the order does
+// not matter), divided in fp64 and rounded once to fp32; every division of
+// the quantisers is an IEEE fp32 division (__fdiv_rn) and the INT8 rounding
+// is round-half-to-even (__float2int_rn).  Do not build with fast-math.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace sage {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kStatRows = 256;  // tokens per CTA in the K/V statistics pass
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&x)[8]);
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <>
+__device__ __forceinline__ void load8<__half>(const __half* p, float (&x)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+    const float2 f = __half22float2(h);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
+// rows of a [r0, r0 + rows) block that lie below N
+__device__ __forceinline__ int rows_valid(int N, int64_t r0, int rows) {
+  const int64_t v = (int64_t)N - r0;
+  return v <= 0 ? 0 : (v < rows ? (int)v : rows);
+}
+
+__device__ __forceinline__ int8_t quant_i8(float x, float s) {
+  if (s == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(x, s));
+  q = q > 127 ? 127 : (q < -127 ? -127 : q);
+  return static_cast<int8_t>(q);
+}
+
+__device__ __forceinline__ uint2 pack8_i8(const int8_t (&c)[8]) {
+  uint2 u;
+  u.x = (uint32_t)(uint8_t)c[0] | ((uint32_t)(uint8_t)c[1] << 8) | ((uint32_t)(uint8_t)c[2] << 16) |
+        ((uint32_t)(uint8_t)c[3] << 24);
+  u.y = (uint32_t)(uint8_t)c[4] | ((uint32_t)(uint8_t)c[5] << 8) | ((uint32_t)(uint8_t)c[6] << 16) |
+        ((uint32_t)(uint8_t)c[7] << 24);
+  return u;
+}
+
+// CTA-wide max of non-negative floats; every thread gets the result.
+__device__ __forceinline__ float block_max_nonneg(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x / 32;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float r = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kThreads / 32; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Pass 1: per (b, kv-head, channel) fp64 sum of K (smooth K) and max |V|.
+// grid (ceil(N / kStatRows), B*Hkv)
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
+  constexpr int CH = D / 8, RG = kThreads / CH;
+  __shared__ double s_sum[kThreads][8];
+  __shared__ float s_amax[kThreads][8];
+  const int bg = blockIdx.y;
+  const int64_t r0 = (int64_t)blockIdx.x * kStatRows;
+  const int64_t r1 = (r0 + kStatRows < (int64_t)a.N) ? r0 + kStatRows : (int64_t)a.N;
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
+  const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)bg * a.N * D;
+  double ks[8];
+  float va[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { ks[e] = 0.0; va[e] = 0.0f; }
+  for (int64_t r = r0 + rg; r < r1; r += RG) {
+    float x[8];
+    load8<T>(K + r * D + ch * 8, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ks[e] += (double)x[e];
+    load8<T>(V + r * D + ch * 8, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) va[e] = fmaxf(va[e], fabsf(x[e]));
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { s_sum[threadIdx.x][e] = ks[e]; s_amax[threadIdx.x][e] = va[e]; }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    double s = 0.0;
+    float m = 0.0f;
+    for (int g = 0; g < RG; ++g) {
+      s += s_sum[g * CH + c / 8][c % 8];
+      m = fmaxf(m, s_amax[g * CH + c / 8][c % 8]);
+    }
+    if (a.smooth_k) atomicAdd(&a.ksum[(int64_t)bg * D + c], s);
+    atomicMax(&a.vamax[(int64_t)bg * D + c], __float_as_uint(m));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Pass 2a: K (bk-row INT8 blocks of gamma(K)) and V (per-channel E4M3,
+// transposed to [d, Np]) for one 128-token tile.  grid (Np/128, B*Hkv)
+template <typename T, int D, int BK>
+__global__ void __launch_bounds__(kThreads) kv_quant_kernel(QuantArgs a) {
+  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, PPB = BK / RG;  // passes per K block
+  constexpr int NKB = kTile / BK;
+  __shared__ float s_km[D], s_sv[D], s_red[kThreads / 32];
+  __shared__ float s_bmax[NKB];
+  __shared__ __align__(16) uint8_t s_vt[D][kTile + 16];
+  const int bg = blockIdx.y, tile = blockIdx.x;
+  const int64_t r0 = (int64_t)tile * kTile;
+  const int valid = rows_valid(a.N, r0, kTile);
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    const float km = a.smooth_k ? __double2float_rn(__ddiv_rn(a.ksum[(int64_t)bg * D + c], (double)a.N)) : 0.0f;
+    const float sv = __fdiv_rn(__uint_as_float(a.vamax[(int64_t)bg * D + c]), 448.0f);
+    s_km[c] = km;
+    s_sv[c] = sv;
+    if (tile == 0) {
+      a.km[(int64_t)bg * D + c] = km;
+      a.s_v[(int64_t)bg * D + c] = sv;
+    }
+  }
+  if (threadIdx.x < NKB) s_bmax[threadIdx.x] = 0.0f;
+  __syncthreads();
+
+  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
+  const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)bg * a.N * D;
+
+  // ---- K: gamma(K) = K - km, per-block amax, INT8 codes
+  float x[NP][8];
+  float bm[NKB];
+#pragma unroll
+  for (int kb = 0; kb < NKB; ++kb) bm[kb] = 0.0f;
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    if (r < valid) {
+      load8<T>(K + (r0 + r) * D + ch * 8, x[p]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[p][e] = __fsub_rn(x[p][e], s_km[ch * 8 + e]);
+        bm[p / PPB] = fmaxf(bm[p / PPB], fabsf(x[p][e]));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[p][e] = 0.0f;
+    }
+  }
+#pragma unroll
+  for (int kb = 0; kb < NKB; ++kb) {
+    const float m = block_max_nonneg(bm[kb], s_red);
+    if (threadIdx.x == 0) s_bmax[kb] = m;
+  }
+  __syncthreads();
+  float sk[NKB];
+#pragma unroll
+  for (int kb = 0; kb < NKB; ++kb) {
+    sk[kb] = __fdiv_rn(s_bmax[kb], 127.0f);
+    const int gb = tile * NKB + kb;
+    if (threadIdx.x == 0 && gb < a.Tn) a.s_k[(int64_t)bg * a.Tn + gb] = sk[kb];
+  }
+  int8_t* k8 = a.k8 + (int64_t)bg * a.Np * D;
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    int8_t c8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], sk[p / PPB]) : (int8_t)0;
+    *reinterpret_cast<uint2*>(k8 + (r0 + r) * D + ch * 8) = pack8_i8(c8);
+  }
+
+  // ---- V: E4M3(V / s_v[c]), transposed through shared memory
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    float v[8];
+    if (r < valid) {
+      load8<T>(V + (r0 + r) * D + ch * 8, v);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float sv0 = s_sv[ch * 8 + e], sv1 = s_sv[ch * 8 + e + 1];
+      const float f0 = (sv0 == 0.0f) ? 0.0f : __fdiv_rn(v[e], sv0);
+      const float f1 = (sv1 == 0.0f) ? 0.0f : __fdiv_rn(v[e + 1], sv1);
+      const uint32_t two = cvt_e4m3x2(f0, f1);
+      s_vt[ch * 8 + e][r] = (uint8_t)(two & 0xFF);
+      s_vt[ch * 8 + e + 1][r] = (uint8_t)(two >> 8);
+    }
+  }
+  __syncthreads();
+  uint8_t* vt = a.v8t + (int64_t)bg * D * a.Np + r0;
+  for (int i = threadIdx.x; i < D * (kTile / 16); i += kThreads) {
+    const int c = i / (kTile / 16), part = i % (kTile / 16);
+    *reinterpret_cast<uint4*>(vt + (int64_t)c * a.Np + part * 16) =
+        *reinterpret_cast<const uint4*>(&s_vt[c][part * 16]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Pass 2b: Q blocks of BQ rows: optional block mean (smooth Q), amax, INT8.
+// grid (Np/BQ, B*Hq)
+template <typename T, int D, int BQ>
+__global__ void __launch_bounds__(kThreads) q_quant_kernel(QuantArgs a) {
+  constexpr int CH = D / 8, RG = kThreads / CH, NP = BQ / RG;
+  __shared__ double s_sum[kThreads][8];
+  __shared__ float s_mean[D], s_red[kThreads / 32];
+  const int bh = blockIdx.y, blk = blockIdx.x;
+  const int64_t r0 = (int64_t)blk * BQ;
+  const int valid = rows_valid(a.N, r0, BQ);
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  int8_t* q8 = a.q8 + (int64_t)bh * a.Np * D;
+
+  if (valid == 0) {  // padding rows between N and Np
+#pragma unroll
+    for (int p = 0; p < NP; ++p)
+      *reinterpret_cast<uint2*>(q8 + (r0 + rg + p * RG) * D + ch * 8) = make_uint2(0u, 0u);
+    return;
+  }
+  const T* Q = reinterpret_cast<const T*>(a.q) + (int64_t)bh * a.N * D;
+  float x[NP][8];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    if (r < valid) {
+      load8<T>(Q + (r0 + r) * D + ch * 8, x[p]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[p][e] = 0.0f;
+    }
+  }
+  if (a.smooth_q) {
+    double cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+    for (int p = 0; p < NP; ++p)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] += (double)x[p][e];  // invalid rows hold 0
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      const int c = threadIdx.x;
+      double s = 0.0;
+      for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
+      const float mu = __double2float_rn(__ddiv_rn(s, (double)valid));
+      s_mean[c] = mu;
+      a.qbar[((int64_t)bh * a.Tm + blk) * D + c] = mu;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int p = 0; p < NP; ++p)
+      if (rg + p * RG < valid)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[p][e] = __fsub_rn(x[p][e], s_mean[ch * 8 + e]);
+  }
+  float am = 0.0f;
+#pragma unroll
+  for (int p = 0; p < NP; ++p)
+    if (rg + p * RG < valid)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x[p][e]));
+  const float amax = block_max_nonneg(am, s_red);
+  const float s = __fdiv_rn(amax, 127.0f);
+  if (threadIdx.x == 0) a.s_q[(int64_t)bh * a.Tm + blk] = s;
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    int8_t c8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], s) : (int8_t)0;
+    *reinterpret_cast<uint2*>(q8 + (r0 + r) * D + ch * 8) = pack8_i8(c8);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Pass 3 (smooth Q): delta_S[b,h,i,j] = sum_c qbar[i,c] * gamma(K)[j,c] for one
+// 128-key tile and every Q block i.  fp32 accumulation in channel order.
+// grid (Np/128, B*Hq); dynamic smem: D*128 floats (gamma^T)
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) delta_s_kernel(QuantArgs a) {
+  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG;
+  extern __shared__ float s_gT[];  // [D][kTile]
+  const int bh = blockIdx.y, tile = blockIdx.x;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const int bg = b * a.Hkv + h / (a.Hq / a.Hkv);
+  const int64_t r0 = (int64_t)tile * kTile;
+  const int valid = rows_valid(a.N, r0, kTile);
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
+  const float* km = a.km + (int64_t)bg * D;
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    float x[8];
+    if (r < valid) {
+      load8<T>(K + (r0 + r) * D + ch * 8, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], km[ch * 8 + e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s_gT[(ch * 8 + e) * kTile + r] = x[e];
+  }
+  __syncthreads();
+  const int key = threadIdx.x % kTile;
+  const float* qb = a.qbar + (int64_t)bh * a.Tm * D;
+  float* out = a.dS + (int64_t)bh * a.Tm * a.Np + r0 + key;
+  for (int i0 = threadIdx.x / kTile; i0 < a.Tm; i0 += 2 * (kThreads / kTile)) {
+    const int i1 = i0 + kThreads / kTile;
+    float acc0 = 0.0f, acc1 = 0.0f;
+    const float* q0 = qb + (int64_t)i0 * D;
+    const float* q1 = qb + (int64_t)min(i1, a.Tm - 1) * D;
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) {
+      const float gv = s_gT[c * kTile + key];
+      acc0 = fmaf(__ldg(q0 + c), gv, acc0);
+      acc1 = fmaf(__ldg(q1 + c), gv, acc1);
+    }
+    out[(int64_t)i0 * a.Np] = acc0;
+    if (i1 < a.Tm) out[(int64_t)i1 * a.Np] = acc1;
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_quant_t(const QuantArgs& a, cudaStream_t st) {
+  cudaError_t e;
+  const int BHkv = a.B * a.Hkv, BHq = a.B * a.Hq;
+  const int kv_tiles = (int)(a.Np / kTile);
+  if (a.smooth_k) {
+    e = cudaMemsetAsync(a.ksum, 0, sizeof(double) * (size_t)BHkv * D, st);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaMemsetAsync(a.vamax, 0, sizeof(unsigned) * (size_t)BHkv * D, st);
+  if (e != cudaSuccess) return e;
+  kv_stats_kernel<T, D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(a);
+  if (a.bk == 64)
+    kv_quant_kernel<T, D, 64><<<dim3(kv_tiles, BHkv), kThreads, 0, st>>>(a);
+  else
+    kv_quant_kernel<T, D, 128><<<dim3(kv_tiles, BHkv), kThreads, 0, st>>>(a);
+  if (a.bq == 64)
+    q_quant_kernel<T, D, 64><<<dim3((int)(a.Np / 64), BHq), kThreads, 0, st>>>(a);
+  else
+    q_quant_kernel<T, D, 128><<<dim3((int)(a.Np / 128), BHq), kThreads, 0, st>>>(a);
+  if (a.smooth_q) {
+    const size_t smem = sizeof(float) * D * kTile;
+    e = cudaFuncSetAttribute(delta_s_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    delta_s_kernel<T, D><<<dim3(kv_tiles, BHq), kThreads, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quant(const QuantArgs& a, int is_fp16, cudaStream_t st) {
+  if (is_fp16) return a.D == 128 ? launch_quant_t<__half, 128>(a, st) : launch_quant_t<__half, 64>(a, st);
+  return a.D == 128 ? launch_quant_t<__nv_bfloat16, 128>(a, st) : launch_quant_t<__nv_bfloat16, 64>(a, st);
+}
+
+}  // namespace sage

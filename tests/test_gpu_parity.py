@@ -1,0 +1,143 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Quantised tensors, scales and INT32 QK^T tiles are
+compared bit-exactly; attention outputs element by element within max-abs
+1e-2 and cosine >= 0.9999."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_attention_block_b200 import sage
+from quantized_attention_block_b200 import workloads as W
+
+from harness import compare_out, compare_quant, gpu_attention, gpu_quant, oracle_quant, oracle_rows
+
+pytestmark = pytest.mark.gpu
+
+# Same recipes at sizes the oracle finishes in seconds: several 128-row tiles
+# and a ragged tail (N % 128 != 0, N % 64 != 0).
+SMALL = {
+    "tiny": W.get("tiny"),
+    "prefill": W.small_variant(W.get("prefill"), N=600, B=1, Hq=2),
+    "video": W.small_variant(W.get("video"), N=600, B=1, Hq=2),
+    "gqa": W.small_variant(W.get("gqa"), N=600, B=1, Hq=8, Hkv=2),
+}
+EDGE = {
+    "N1": W.get("tiny").with_(name="N1", N=1, bq=128),
+    "N127_causal": W.get("prefill").with_(name="N127_causal", B=1, Hq=1, Hkv=1, N=127),
+    "N129_causal_d64": W.get("video").with_(name="N129_causal_d64", B=1, Hq=2, Hkv=2, N=129, causal=True),
+    "N200_fp16_bq64_bk128": W.get("tiny").with_(name="N200_fp16", N=200, bq=64, bk=128),
+    "N300_no_smooth_k": W.get("prefill").with_(name="N300_nosk", B=2, Hq=2, Hkv=1, N=300, smooth_k=False),
+    "N257_smoothq_causal_d128": W.get("gqa").with_(name="N257_sq", B=1, Hq=2, Hkv=2, N=257, smooth_q=True,
+                                                   qk_shared_bias_std=2.0, k_bias_std=0.0),
+    "N513_bq64_bk64_d64": W.get("video").with_(name="N513", B=1, Hq=1, Hkv=1, N=513, bq=64),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL) + list(EDGE))
+def test_quant_bit_exact(name):
+    w = {**SMALL, **EDGE}[name]
+    q, k, v = W.make_qkv(w)
+    p, ws, view, _ = gpu_quant(w, q, k, v)
+    bad = compare_quant(w, p, ws, view, oracle_quant(w, q, k, v))
+    assert not bad, bad
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill", "video", "gqa"])
+def test_qk_int32_tiles_bit_exact(name):
+    w = SMALL[name]
+    q, k, v = W.make_qkv(w)
+    p, ws, view, _ = gpu_quant(w, q, k, v)
+    t = sage.view_tensors(view, p, ws)
+    q8 = t["q8"].cpu().numpy().astype(np.int64)
+    k8 = t["k8"].cpu().numpy().astype(np.int64)
+    G = w.Hq // w.Hkv
+    ntile = int(view.Np) // 128
+    for (b, h, qt, kt) in [(0, 0, 0, 0), (0, w.Hq - 1, ntile - 1, 0), (w.B - 1, w.Hq // 2, 0, ntile - 1),
+                           (0, 0, ntile - 1, ntile - 1)]:
+        got = sage.sage_debug_qk_int32(view, p, b, h, qt, kt).cpu().numpy()
+        ref = q8[b, h, qt * 128:(qt + 1) * 128] @ k8[b, h // G, kt * 128:(kt + 1) * 128].T
+        np.testing.assert_array_equal(got, ref.astype(np.int32))
+
+
+@pytest.mark.parametrize("name", list(SMALL) + list(EDGE))
+def test_attention_matches_oracle_elementwise(name):
+    w = {**SMALL, **EDGE}[name]
+    q, k, v = W.make_qkv(w)
+    p, ws, view, o = gpu_attention(w, q, k, v)
+    quant = oracle_quant(w, q, k, v)
+    out = o.float().cpu().numpy()
+    refs = np.stack([np.stack([oracle_rows(w, quant, b, h, 0, w.N) for h in range(w.Hq)]) for b in range(w.B)])
+    m, ok = compare_out(refs, out)
+    assert ok, m
+
+
+def test_sage_attn_fwd_one_call_equals_two_step():
+    w = SMALL["prefill"]
+    q, k, v = W.make_qkv(w)
+    _, _, _, o2 = gpu_attention(w, q, k, v)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o1 = sage.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                            smooth_q=w.smooth_q, bq=w.bq, bk=w.bk)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """Failure detection without a fault: a wait nobody ends gives up after the
+    limit, the status comes back as SAGE_ERR_TIMEOUT, and the context still works."""
+    assert sage.sage_last_device_error() == 0
+    assert sage.sage_debug_bounded_wait(2000) == 7  # SAGE_ERR_TIMEOUT
+    assert sage.sage_last_device_error() == 0       # cleared
+    w = SMALL["tiny"]
+    q, k, v = W.make_qkv(w)
+    gpu_attention(w, q, k, v)
+
+
+def test_rejects_non_sm100_inputs_cleanly():
+    w = SMALL["tiny"]
+    q, k, v = W.make_qkv(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    with pytest.raises(sage.SageError):
+        sage.sage_attn_fwd(qd, kd, vd, bq=96)
+    with pytest.raises(sage.SageError):
+        sage.sage_attn_fwd(qd[..., :48].contiguous(), kd[..., :48].contiguous(), vd[..., :48].contiguous())
+
+
+# ---------------------------------------------------------------- full sizes
+FULL = ["prefill", "video", "gqa"]
+
+
+def _sample_tiles(n_tiles, rng, k=3):
+    picks = {0, n_tiles - 1}
+    while len(picks) < min(n_tiles, k + 2):
+        picks.add(int(rng.integers(0, n_tiles)))
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_quant_bit_exact_and_sampled_attention(name):
+    """At the benchmark's sizes and launch configuration: every quantised value
+    checked bit-exactly; attention outputs on sampled Q tiles of sampled heads
+    (first, last / ragged tail, random) checked element by element."""
+    w = W.get(name)
+    q, k, v = W.make_qkv(w)
+    p, ws, view, o = gpu_attention(w, q, k, v)
+    quant = oracle_quant(w, q, k, v)
+    bad = compare_quant(w, p, ws, view, quant)
+    assert not bad, bad
+    rng = np.random.default_rng(123)
+    n_tiles = int(view.Np) // 128
+    heads = sorted({(0, 0), (w.B - 1, w.Hq - 1), (int(rng.integers(0, w.B)), int(rng.integers(0, w.Hq)))})
+    from concurrent.futures import ThreadPoolExecutor
+    jobs = []
+    for (b, h) in heads:
+        for t in _sample_tiles(n_tiles, rng, k=2):
+            r0, r1 = t * 128, min((t + 1) * 128, w.N)
+            jobs.append((b, h, r0, r1))
+    with ThreadPoolExecutor() as ex:
+        refs = list(ex.map(lambda j: oracle_rows(w, quant, *j), jobs))
+    out = o.float().cpu().numpy()
+    for (b, h, r0, r1), ref in zip(jobs, refs):
+        m, ok = compare_out(ref, out[b, h, r0:r1])
+        assert ok, ((b, h, r0, r1), m)
