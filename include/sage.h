@@ -151,6 +151,35 @@ SAGE_API sage_status sage_last_device_error(void *stream);
  */
 SAGE_API sage_status sage_debug_bounded_wait(uint32_t timeout_us, void *stream);
 
+/*
+ * Size of the device scratch array that sage_attn_fwd_noalloc uses (32 MiB).
+ * Every GPU that loads this library reserves it until the process exits.
+ */
+#define SAGE_STATIC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * sage_attn_fwd without a workspace argument.  The method has no counterpart
+ * for this: it exists for callers that cannot allocate device memory at all
+ * (a plugin interface that only hands over input and output pointers, or a
+ * process whose device memory is owned by another allocator), so cudaMalloc
+ * is not open to them.  It computes exactly what sage_attn_fwd computes, with
+ * its scratch in a fixed library-owned device array of
+ * SAGE_STATIC_SCRATCH_BYTES bytes instead of a caller workspace.
+ *   - q, k, v, o: device pointers as for sage_attn_fwd (caller-owned).
+ *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library
+ *     routine.
+ *   - Returns SAGE_ERR_WORKSPACE_TOO_SMALL when sage_workspace_bytes(p)
+ *     exceeds SAGE_STATIC_SCRATCH_BYTES (nothing is enqueued then).
+ *   - The first call on a device looks up the array's device address on
+ *     that device (the device must be current) and caches it; make that first
+ *     call before any stream capture.
+ *   - All calls on a device share the one array, and it keeps whatever the
+ *     last call left in it.  Calls whose work overlaps on the GPU (different
+ *     streams, or host threads without ordering) race on it; order them.
+ */
+SAGE_API sage_status sage_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *o,
+                                           const sage_params *p, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 SAGE_API const char *sage_status_string(sage_status s);
 

@@ -4,3 +4,4 @@
 #include "quant.cu"
 #include "attn_i8f8.cu"
 #include "api.cu"
+#include "noalloc.cu"

@@ -25,7 +25,7 @@ STATUS_NAMES = {
 }
 EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd",
             "sage_debug_qk_int32", "sage_last_device_error", "sage_debug_bounded_wait",
-            "sage_status_string")
+            "sage_status_string", "sage_attn_fwd_noalloc")
 
 
 class SageError(RuntimeError):
@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.sage_last_device_error.argtypes = [vp]
         L.sage_debug_bounded_wait.argtypes = [ctypes.c_uint32, vp]
         L.sage_status_string.argtypes, L.sage_status_string.restype = [ctypes.c_int], ctypes.c_char_p
+        L.sage_attn_fwd_noalloc.argtypes, L.sage_attn_fwd_noalloc.restype = [vp, vp, vp, vp, P, vp], ctypes.c_int
         for n in ("sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd", "sage_debug_qk_int32",
                   "sage_last_device_error", "sage_debug_bounded_wait"):
             getattr(L, n).restype = ctypes.c_int
