@@ -10,19 +10,24 @@
 //   P~_ij = exp(S_ij - m_ij),   l_ij = e^(m_i,j-1 - m_ij) l_i,j-1 + rowsum P~_ij
 //   O_t   = E4M3(448 P~_ij) V^_j                  FP8 MMA (kind::f8f6f4) into a
 //                                                 fresh TMEM tile (level 1)
-//   O     = e^(m_i,j-1 - m_ij) O + O_t             FP32 in registers (level 2)
+//   O     = e^(m_i,j-1 - m_ij) O + O_t             FP32 on CUDA cores (level 2)
 //   out   = O / l / 448 * delta_V
 // The exponentials run in base 2 (scores pre-multiplied by log2 e); the 448
 // is folded into the exponent (exp2(t - m + log2 448)), so l accumulates
 // 448 P~ and the final division by l absorbs the /448.
 //
-// CTA = one (batch, head, Q tile); 192 threads in three roles:
-//   warp 0      TMA producer: Q tile once, then K_j / V_j^T into a 2-stage ring
-//   warp 1      MMA issuer (one thread) and TMEM owner (whole warp)
-//   warps 2..5  softmax + correction + epilogue; thread = one Q row = one TMEM lane
-// TMEM columns: [0, 128) S (int32), [128, 128 + D) O_t (fp32).
-// P goes through shared memory in the 128-byte-swizzled K-major layout the
-// MMA reads (the same layout TMA writes for K and V^T).
+// CTA = one (batch, head) and TWO consecutive 128-row Q tiles that share every
+// K / V tile.  512 threads in four warpgroups:
+//   WG0  warp 0: TMA producer (Q tiles once, K_j / V_j^T through a ring)
+//        warp 1: MMA issuer (one thread) and TMEM owner; warps 2-3 idle
+//   WG1  softmax of Q tile 0    (thread = one Q row = one TMEM lane)
+//   WG2  softmax of Q tile 1
+//   WG3  level-2 accumulation O = alpha O + O_t for both tiles, and the epilogue
+// The two softmax warpgroups take turns (ping-pong on mbarriers), so the MMA
+// and correction chain of one tile runs while the other tile's softmax owns
+// the issue slots.  TMEM (512 columns): tile i's S_i / O_t_i share columns
+// [128 i, 128 i + 128) (P goes through shared memory, so S is dead once the
+// softmax has read it); O_i lives at [256 + D i, 256 + D (i + 1)).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -33,9 +38,13 @@ namespace sage {
 
 namespace {
 
-constexpr int kStages = 2;
-constexpr int kThreadsAttn = 192;
+constexpr int kStages = 3;
+constexpr int kThreadsAttn = 512;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
+
+// per-warpgroup register budgets after setmaxnreg (sum x 128 <= 65536)
+constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 176, kRegsCorrection = 104;
+static_assert(kRegsProducer + 2 * kRegsSoftmax + kRegsCorrection <= 512, "register split exceeds the launch");
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -44,12 +53,14 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 template <int D>
 struct Smem {
   static constexpr uint32_t kQ = 128 * D, kK = 128 * D, kV = D * 128, kP = 128 * 128;
-  static constexpr uint32_t oQ = 0;
-  static constexpr uint32_t oK = oQ + kQ;
-  static constexpr uint32_t oV = oK + kStages * kK;
-  static constexpr uint32_t oP = oV + kStages * kV;
-  static constexpr uint32_t oBar = oP + kP;
-  static constexpr uint32_t kNumBars = 1 + 3 * kStages + 4;
+  static constexpr uint32_t oQ = 0;                      // 2 tiles
+  static constexpr uint32_t oK = oQ + 2 * kQ;            // kStages
+  static constexpr uint32_t oV = oK + kStages * kK;      // kStages
+  static constexpr uint32_t oP = oV + kStages * kV;      // 2 tiles
+  static constexpr uint32_t oAlpha = oP + 2 * kP;        // float[2][128]
+  static constexpr uint32_t oL = oAlpha + 2 * 128 * 4;   // float[2][128]
+  static constexpr uint32_t oBar = oL + 2 * 128 * 4;
+  static constexpr uint32_t kNumBars = 1 + 3 * kStages + 6 * 2;
   static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = oTmem + 16 + 1024;  // + alignment slack
 };
@@ -67,6 +78,19 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+struct Bars {
+  uint64_t* q_full;
+  uint64_t* k_full;    // [kStages]
+  uint64_t* v_full;    // [kStages]
+  uint64_t* kv_empty;  // [kStages]
+  uint64_t* s_full;    // [2]  QK^T of tile i done            (tcgen05.commit)
+  uint64_t* p_full;    // [2]  P_i and alpha_i written         (128 softmax threads)
+  uint64_t* ot_full;   // [2]  O_t of tile i done              (tcgen05.commit)
+  uint64_t* r_free;    // [2]  O_t_i consumed, columns free    (128 correction threads)
+  uint64_t* turn;      // [2]  softmax ping-pong: tile i may run (128 threads of the other tile)
+  uint64_t* l_ready;   // [2]  final l of tile i in shared memory
+};
+
 template <int D, bool CAUSAL, bool HAS_DS, typename TO>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -76,7 +100,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   constexpr uint32_t kSboQK = 8 * D;  // 8 rows x D bytes per swizzle atom
   constexpr uint32_t kIdescQK = make_idesc(/*S32*/ 2, /*s8*/ 1, /*s8*/ 1, 128, 128);
   constexpr uint32_t kIdescPV = make_idesc(/*F32*/ 1, /*E4M3*/ 0, /*E4M3*/ 0, 128, D);
-  constexpr uint32_t kTmemCols = 256;
+  constexpr uint32_t kTmemCols = 512;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -84,37 +108,55 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* sK = smem + L::oK;
   uint8_t* sV = smem + L::oV;
   uint8_t* sP = smem + L::oP;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::oBar);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + kStages;
-  uint64_t* kv_empty = v_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_free + 1;
-  uint64_t* pv_done = p_full + 1;
+  float* s_alpha = reinterpret_cast<float*>(smem + L::oAlpha);
+  float* s_l = reinterpret_cast<float*>(smem + L::oL);
+  uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L::oBar);
+  Bars bar;
+  bar.q_full = bar0;
+  bar.k_full = bar0 + 1;
+  bar.v_full = bar.k_full + kStages;
+  bar.kv_empty = bar.v_full + kStages;
+  bar.s_full = bar.kv_empty + kStages;
+  bar.p_full = bar.s_full + 2;
+  bar.ot_full = bar.p_full + 2;
+  bar.r_free = bar.ot_full + 2;
+  bar.turn = bar.r_free + 2;
+  bar.l_ready = bar.turn + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oTmem);
 
-  // heavy (long causal) tiles first
+  // ---- work: (b, h, pair of Q tiles), heavy causal pairs first
   const int bhq = a.B * a.Hq;
-  const int qtile = a.n_qtiles - 1 - (int)(blockIdx.x / bhq);
+  const int n_pairs = (a.n_qtiles + 1) / 2;
+  const int pr = n_pairs - 1 - (int)(blockIdx.x / bhq);
   const int bh = blockIdx.x % bhq;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const int g = h / (a.Hq / a.Hkv);
-  const int nT = CAUSAL ? qtile + 1 : (int)(a.Np / kTile);
+  const int n_kt = (int)(a.Np / kTile);
+  int nTi[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int qt = 2 * pr + i;
+    nTi[i] = qt >= a.n_qtiles ? 0 : (CAUSAL ? qt + 1 : n_kt);
+  }
+  const int nT = nTi[0] > nTi[1] ? nTi[0] : nTi[1];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int wg = warp / 4;
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(bar.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.kv_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.s_full[i], 1);
+      mbar_init(&bar.p_full[i], 128);
+      mbar_init(&bar.ot_full[i], 1);
+      mbar_init(&bar.r_free[i], 128);
+      mbar_init(&bar.turn[i], 128);
+      mbar_init(&bar.l_ready[i], 128);
+    }
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -125,194 +167,255 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (wg == 0) {
+    regs_dec<kRegsProducer>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ TMA producer
       tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
-      const int qrow = (int)((int64_t)(b * a.Hq + h) * a.Np + (int64_t)qtile * kTile);
+      const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
       const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np);
       const int vrow = (b * a.Hkv + g) * D;
-      mbar_expect_tx(q_full, L::kQ);
-      tma_load_2d(sQ, &tmQ, q_full, 0, qrow);
+      mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
+      for (int i = 0; i < 2; ++i)
+        if (nTi[i] > 0) tma_load_2d(sQ + i * L::kQ, &tmQ, bar.q_full, 0, (int)(qhead + (int64_t)(2 * pr + i) * kTile));
       bool ok = true;
       int j = 0;
       for (; j < nT && ok; ++j) {
         const int s = j % kStages;
-        if (j >= kStages) ok = mbar_wait(&kv_empty[s], ((j / kStages) + 1) & 1);
+        if (j >= kStages) ok = mbar_wait(&bar.kv_empty[s], ((j / kStages) + 1) & 1);
         if (!ok) break;
-        mbar_expect_tx(&k_full[s], L::kK);
-        tma_load_2d(sK + s * L::kK, &tmK, &k_full[s], 0, krow0 + j * kTile);
-        mbar_expect_tx(&v_full[s], L::kV);
-        tma_load_2d(sV + s * L::kV, &tmV, &v_full[s], j * kTile, vrow);
+        mbar_expect_tx(&bar.k_full[s], L::kK);
+        tma_load_2d(sK + s * L::kK, &tmK, &bar.k_full[s], 0, krow0 + j * kTile);
+        mbar_expect_tx(&bar.v_full[s], L::kV);
+        tma_load_2d(sV + s * L::kV, &tmV, &bar.v_full[s], j * kTile, vrow);
       }
-      // never leave a copy in flight: wait for the last loads to land
-      for (int jj = max(0, j - kStages); jj < j; ++jj) {
-        mbar_wait(&k_full[jj % kStages], (jj / kStages) & 1);
-        mbar_wait(&v_full[jj % kStages], (jj / kStages) & 1);
+      // never leave a copy in flight
+      for (int jj = (j - kStages > 0 ? j - kStages : 0); jj < j; ++jj) {
+        mbar_wait(&bar.k_full[jj % kStages], (jj / kStages) & 1);
+        mbar_wait(&bar.v_full[jj % kStages], (jj / kStages) & 1);
       }
-      mbar_wait(q_full, 0);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0);
-      int issued_pv = 0;
-      auto issue_pv = [&](int jj) -> bool {
-        const int s = jj % kStages;
-        if (!mbar_wait(p_full, jj & 1)) return false;
-        if (!mbar_wait(&v_full[s], (jj / kStages) & 1)) return false;
-        tc_fence_after();
-        const uint32_t aV = smem_u32(sV + s * L::kV);
+      mbar_wait(bar.q_full, 0);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t aP0 = smem_u32(sP);
+        bool ok = mbar_wait(bar.q_full, 0);
+        uint32_t last_ot[2] = {0, 0}, last_s[2] = {0, 0};  // commits per tile
+        auto issue_qk = [&](int i, int j) {
+          const int s = j % kStages;
+          const uint32_t aQ = smem_u32(sQ + i * L::kQ), aK = smem_u32(sK + s * L::kK);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 32; ++kk)
-          mma_f8f6f4(tO, make_sdesc(aP + kk * 32, 1024, kSwizzle128B), make_sdesc(aV + kk * 32, 1024, kSwizzle128B),
-                     kIdescPV, kk > 0 ? 1u : 0u);
-        mma_commit(pv_done);
-        mma_commit(&kv_empty[s]);
-        ++issued_pv;
-        return true;
-      };
-      for (int j = 0; j < nT && ok; ++j) {
-        const int s = j % kStages;
-        ok = mbar_wait(&k_full[s], (j / kStages) & 1);
-        if (ok && j > 0) ok = mbar_wait(s_free, (j - 1) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t aK = smem_u32(sK + s * L::kK);
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_i8(tmem + 128 * i, make_sdesc(aQ + kk * 32, kSboQK, kSwzQK), make_sdesc(aK + kk * 32, kSboQK, kSwzQK),
+                   kIdescQK, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.s_full[i]);
+          ++last_s[i];
+        };
+        auto issue_pv = [&](int i, int j) {
+          const int s = j % kStages;
+          const uint32_t aP = aP0 + i * L::kP, aV = smem_u32(sV + s * L::kV);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8(tS, make_sdesc(aQ + kk * 32, kSboQK, kSwzQK), make_sdesc(aK + kk * 32, kSboQK, kSwzQK), kIdescQK,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-        if (j > 0) ok = issue_pv(j - 1);
+          for (int kk = 0; kk < kTile / 32; ++kk)
+            mma_f8f6f4(tmem + 128 * i, make_sdesc(aP + kk * 32, 1024, kSwizzle128B),
+                       make_sdesc(aV + kk * 32, 1024, kSwizzle128B), kIdescPV, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.ot_full[i]);
+          ++last_ot[i];
+        };
+        if (ok) ok = mbar_wait(&bar.k_full[0], 0);
+        if (ok) {
+          tc_fence_after();
+          for (int i = 0; i < 2; ++i)
+            if (nTi[i] > 0) issue_qk(i, 0);
+        }
+        for (int j = 0; j < nT && ok; ++j) {
+          const int s = j % kStages;
+          if (!(ok = mbar_wait(&bar.v_full[s], (j / kStages) & 1))) break;
+          bool k_next = false;
+          for (int i = 0; i < 2 && ok; ++i) {
+            if (j < nTi[i]) {
+              if (!(ok = mbar_wait(&bar.p_full[i], j & 1))) break;
+              tc_fence_after();
+              issue_pv(i, j);
+            }
+            if (j + 1 < nTi[i]) {
+              if (!k_next) {
+                if (!(ok = mbar_wait(&bar.k_full[(j + 1) % kStages], ((j + 1) / kStages) & 1))) break;
+                k_next = true;
+              }
+              if (!(ok = mbar_wait(&bar.r_free[i], j & 1))) break;
+              tc_fence_after();
+              issue_qk(i, j + 1);
+            }
+          }
+          mma_commit(&bar.kv_empty[s]);
+        }
+        // every tensor-core op retired before TMEM is released
+        for (int i = 0; i < 2; ++i) {
+          if (last_s[i] > 0) mbar_wait(&bar.s_full[i], (last_s[i] - 1) & 1);
+          if (last_ot[i] > 0) mbar_wait(&bar.ot_full[i], (last_ot[i] - 1) & 1);
+        }
       }
-      if (ok) ok = issue_pv(nT - 1);
-      // all tensor-core work retired before the CTA frees TMEM
-      if (issued_pv > 0) mbar_wait(pv_done, (issued_pv - 1) & 1);
+      __syncwarp();
     }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax / correction
+  } else if (wg == 1 || wg == 2) {
+    // ------------------------------------------------------------ softmax
+    regs_inc<kRegsSoftmax>();
+    const int ti = wg - 1;  // Q tile of this warpgroup
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const int qtile = 2 * pr + ti;
     const int64_t qrow = (int64_t)qtile * kTile + row;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + 128 * ti + ((uint32_t)(quarter * 32) << 16);
     const int qblk = min((int)(qrow / a.bq), a.Tm - 1);
     const float row_scale = a.s_q[(int64_t)(b * a.Hq + h) * a.Tm + qblk] * a.scale_log2;
     const float* sk = a.s_k + (int64_t)(b * a.Hkv + g) * a.Tn;
     const float* dsr = HAS_DS ? a.dS + ((int64_t)(b * a.Hq + h) * a.Tm + qblk) * a.Np : nullptr;
-
-    float o[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) o[c] = 0.0f;
-    float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+    uint8_t* myP = sP + ti * L::kP + row * 128;
+    float m = -INFINITY, l = 0.0f;
     bool ok = true;
-    uint32_t r[32];
 
     for (int j = 0; j < nT && ok; ++j) {
-      if (!(ok = mbar_wait_warp(s_full, j & 1))) break;
-      tc_fence_after();
-      const int col0 = j * kTile;
-      float ak[4];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) ak[c4] = row_scale * __ldg(sk + min((col0 + c4 * 32) / a.bk, a.Tn - 1));
-      const bool need_mask = (col0 + kTile > a.N) || (CAUSAL && col0 + kTile - 1 > qtile * kTile);
-
-      // pass 1: row max of this tile (log2 units)
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        tmem_ld32(tS + lane_off + c4 * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = col0 + c4 * 32 + e;
-          float t = (float)(int)r[e] * ak[c4];
-          if (HAS_DS) t = fmaf(__ldg(dsr + col), a.scale_log2, t);
-          const bool masked = need_mask && (col >= a.N || (CAUSAL && col > qrow));
-          if (!masked) mx = fmaxf(mx, t);
-        }
-      }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
-      const float mm = (m_new == -INFINITY) ? 0.0f : m_new - kLog2_448;
-
-      // level-2 accumulation of the previous tile: O = alpha_{j-1} O + O_t
-      if (j > 0) {
-        if (!(ok = mbar_wait_warp(pv_done, (j - 1) & 1))) break;
+      // ping-pong: tile 0 runs iteration j after tile 1 finished j-1; tile 1 after tile 0 finished j
+      if (ti == 0 && j > 0) ok = mbar_wait_warp(&bar.turn[0], (j - 1) & 1);
+      if (ti == 1) ok = ok && mbar_wait_warp(&bar.turn[1], j & 1);
+      if (!ok) break;
+      if (j < nTi[ti]) {
+        if (!(ok = mbar_wait_warp(&bar.s_full[ti], j & 1))) break;
         tc_fence_after();
-#pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4) {
-          tmem_ld32(tO + lane_off + c4 * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[c4 * 32 + e] = fmaf(o[c4 * 32 + e], alpha_prev, __uint_as_float(r[e]));
-        }
-      }
-
-      // pass 2: P = exp2(t - m + log2 448) -> E4M3 -> shared memory (SW128 K-major)
-      float rs = 0.0f;
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        tmem_ld32(tS + lane_off + c4 * 32, r);
+        uint32_t s[128];
+        tmem_ld32p(tS + 0, s + 0);
+        tmem_ld32p(tS + 32, s + 32);
+        tmem_ld32p(tS + 64, s + 64);
+        tmem_ld32p(tS + 96, s + 96);
+        const int col0 = j * kTile;
+        const float a_lo = row_scale * __ldg(sk + min(col0 / a.bk, a.Tn - 1));
+        const float a_hi = row_scale * __ldg(sk + min((col0 + 64) / a.bk, a.Tn - 1));
         tmem_ld_wait();
-        float p[32];
+        // S region is now free for O_t (the MMA overwrites it after p_full)
+        // t = float(acc) * a (+ delta_S * sm_scale * log2 e), in place (as float bits)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = col0 + c4 * 32 + e;
-          float t = (float)(int)r[e] * ak[c4];
-          if (HAS_DS) t = fmaf(__ldg(dsr + col), a.scale_log2, t);
-          const bool masked = need_mask && (col >= a.N || (CAUSAL && col > qrow));
-          p[e] = masked ? 0.0f : ex2_approx(t - mm);
-          rs += p[e];
+        for (int c = 0; c < 128; c += 2) {
+          const float sc = c < 64 ? a_lo : a_hi;
+          float2 x = make_float2(magic_bits_to_float(s[c]), magic_bits_to_float(s[c + 1]));
+          x = fadd2(x, make_float2(-kMagic, -kMagic));  // exact
+          float2 t;
+          if (HAS_DS) {
+            const float2 ds = __ldg(reinterpret_cast<const float2*>(dsr + col0 + c));
+            t = ffma2(x, make_float2(sc, sc), fmul2(ds, make_float2(a.scale_log2, a.scale_log2)));
+          } else {
+            t = fmul2(x, make_float2(sc, sc));
+          }
+          s[c] = __float_as_uint(t.x);
+          s[c + 1] = __float_as_uint(t.y);
         }
+        const bool need_mask = (col0 + kTile > a.N) || (CAUSAL && j == qtile);
+        if (need_mask) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint4 w;
-          w.x = cvt_e4m3x2(p[hh * 16 + 0], p[hh * 16 + 1]) | (cvt_e4m3x2(p[hh * 16 + 2], p[hh * 16 + 3]) << 16);
-          w.y = cvt_e4m3x2(p[hh * 16 + 4], p[hh * 16 + 5]) | (cvt_e4m3x2(p[hh * 16 + 6], p[hh * 16 + 7]) << 16);
-          w.z = cvt_e4m3x2(p[hh * 16 + 8], p[hh * 16 + 9]) | (cvt_e4m3x2(p[hh * 16 + 10], p[hh * 16 + 11]) << 16);
-          w.w = cvt_e4m3x2(p[hh * 16 + 12], p[hh * 16 + 13]) | (cvt_e4m3x2(p[hh * 16 + 14], p[hh * 16 + 15]) << 16);
-          const int chunk = c4 * 2 + hh;
-          *reinterpret_cast<uint4*>(sP + row * 128 + ((chunk ^ (row & 7)) << 4)) = w;
+          for (int c = 0; c < 128; ++c) {
+            const int col = col0 + c;
+            if (col >= a.N || (CAUSAL && col > qrow)) s[c] = __float_as_uint(-INFINITY);
+          }
         }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) mx = fmax3(mx, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        const float m_new = fmaxf(m, mx);
+        const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
+        const float mm = (m_new == -INFINITY) ? 0.0f : m_new - kLog2_448;
+        // P = exp2(t - m + log2 448) -> E4M3 -> shared memory (128B-swizzled K-major)
+        float2 rs2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int grp = 0; grp < 8; ++grp) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            const int c = grp * 16 + e;
+            const float2 u0 = fadd2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                    make_float2(-mm, -mm));
+            const float2 u1 = fadd2(make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])),
+                                    make_float2(-mm, -mm));
+            const float2 p0 = make_float2(ex2_approx(u0.x), ex2_approx(u0.y));
+            const float2 p1 = make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
+            rs2 = fadd2(rs2, fadd2(p0, p1));
+            w[e / 4] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
+          }
+          *reinterpret_cast<uint4*>(myP + ((grp ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        s_alpha[ti * 128 + row] = alpha;
+        tc_fence_before();
+        fence_proxy_async_smem();
+        mbar_arrive(&bar.p_full[ti]);
+        l = fmaf(l, alpha, rs2.x + rs2.y);
+        m = m_new;
       }
-      tc_fence_before();
-      mbar_arrive(s_free);
-      fence_proxy_async_smem();
-      mbar_arrive(p_full);
-      l = fmaf(l, alpha, rs);
-      alpha_prev = alpha;
-      m = m_new;
+      mbar_arrive(&bar.turn[ti ^ 1]);
     }
-
-    if (ok && nT > 0 && (ok = mbar_wait_warp(pv_done, (nT - 1) & 1))) {
-      tc_fence_after();
+    s_l[ti * 128 + row] = l;
+    mbar_arrive(&bar.l_ready[ti]);
+  } else {
+    // ------------------------------------------------------------ correction + epilogue
+    regs_dec<kRegsCorrection>();
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    uint32_t x[32], y[32];
+    for (int j = 0; j < nT && ok; ++j) {
+      for (int i = 0; i < 2; ++i) {
+        if (j >= nTi[i]) continue;
+        if (!(ok = mbar_wait_warp(&bar.ot_full[i], j & 1))) break;
+        if (!(ok = mbar_wait_warp(&bar.p_full[i], j & 1))) break;
+        tc_fence_after();
+        const float alpha = s_alpha[i * 128 + row];
+        const uint32_t tOt = tmem + 128 * i + lane_off, tO = tmem + 256 + D * i + lane_off;
 #pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        tmem_ld32(tO + lane_off + c4 * 32, r);
-        tmem_ld_wait();
+        for (int c = 0; c < D; c += 32) {
+          tmem_ld32(tOt + c, x);
+          if (j > 0) tmem_ld32(tO + c, y);
+          tmem_ld_wait();
+          if (j > 0) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[c4 * 32 + e] = fmaf(o[c4 * 32 + e], alpha_prev, __uint_as_float(r[e]));
+            for (int e = 0; e < 32; e += 2) {
+              const float2 o = ffma2(make_float2(__uint_as_float(y[e]), __uint_as_float(y[e + 1])),
+                                     make_float2(alpha, alpha),
+                                     make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])));
+              x[e] = __float_as_uint(o.x);
+              x[e + 1] = __float_as_uint(o.y);
+            }
+          }
+          tmem_st32(tO + c, x);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar.r_free[i]);
       }
-      // epilogue: out = O / l * delta_V   (l carries the 448)
-      if (qrow < a.N) {
-        const float inv_l = 1.0f / l;
-        const float* sv = a.s_v + (int64_t)(b * a.Hkv + g) * D;
-        TO* out = reinterpret_cast<TO*>(a.o) + ((int64_t)(b * a.Hq + h) * a.N + qrow) * D;
+    }
+    // epilogue: out = O / l * delta_V   (l carries the 448)
+    for (int i = 0; i < 2 && ok; ++i) {
+      if (nTi[i] == 0) continue;
+      if (!(ok = mbar_wait_warp(&bar.l_ready[i], 0))) break;
+      tc_fence_after();
+      const float inv_l = 1.0f / s_l[i * 128 + row];
+      const int64_t qrow = (int64_t)(2 * pr + i) * kTile + row;
+      const float* sv = a.s_v + (int64_t)(b * a.Hkv + g) * D;
+      TO* out = reinterpret_cast<TO*>(a.o) + ((int64_t)(b * a.Hq + h) * a.N + qrow) * D;
+      const uint32_t tO = tmem + 256 + D * i + lane_off;
 #pragma unroll
-        for (int c = 0; c < D; c += 8) {
-          uint4 w;
-          w.x = pack2<TO>(o[c + 0] * inv_l * __ldg(sv + c + 0), o[c + 1] * inv_l * __ldg(sv + c + 1));
-          w.y = pack2<TO>(o[c + 2] * inv_l * __ldg(sv + c + 2), o[c + 3] * inv_l * __ldg(sv + c + 3));
-          w.z = pack2<TO>(o[c + 4] * inv_l * __ldg(sv + c + 4), o[c + 5] * inv_l * __ldg(sv + c + 5));
-          w.w = pack2<TO>(o[c + 6] * inv_l * __ldg(sv + c + 6), o[c + 7] * inv_l * __ldg(sv + c + 7));
-          *reinterpret_cast<uint4*>(out + c) = w;
+      for (int c = 0; c < D; c += 32) {
+        tmem_ld32(tO + c, x);
+        tmem_ld_wait();
+        if (qrow < a.N) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(x[e + u]) * inv_l * __ldg(sv + c + e + u);
+            *reinterpret_cast<uint4*>(out + c + e) =
+                make_uint4(pack2<TO>(f[0], f[1]), pack2<TO>(f[2], f[3]), pack2<TO>(f[4], f[5]), pack2<TO>(f[6], f[7]));
+          }
         }
       }
     }
@@ -416,7 +519,8 @@ cudaError_t launch_attn_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUten
   const int smem = (int)Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)a.n_qtiles * (unsigned)(a.B * a.Hq);
+  const unsigned n_pairs = (unsigned)(a.n_qtiles + 1) / 2;
+  const unsigned grid = n_pairs * (unsigned)(a.B * a.Hq);
   kern<<<grid, kThreadsAttn, smem, st>>>(tmQ, tmK, tmV, a);
   return cudaGetLastError();
 }
