@@ -16,6 +16,7 @@ scaling, no collective on the data path); time = max over ranks.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import json
 import math
 import os
@@ -52,57 +53,76 @@ def _dist():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """Samples SM clock, power and clock-event (throttle) reasons through NVML
+    every few milliseconds while the timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
-        self.proc = None
-        self.path = None
+    def __init__(self, torch_device: int, period_s: float = 0.002):
+        self.dev = torch_device
+        self.period = period_s
+        self.samples = []
+        self.err = None
+        self._stop = None
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            # match the torch device to an NVML device by PCI domain/bus/device numbers
+            props = torch.cuda.get_device_properties(self.dev)
+            self.h = None
+            for idx in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+                info = pynvml.nvmlDeviceGetPciInfo(h)
+                if (int(info.bus), int(info.device), int(info.domain)) == (
+                        int(getattr(props, "pci_bus_id", -1)), int(getattr(props, "pci_device_id", -1)),
+                        int(getattr(props, "pci_domain_id", -1))):
+                    self.h = h
+                    break
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+        except Exception as e:  # pragma: no cover
+            self.err = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            nv = self.nv
+            while not self._stop.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    try:
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    except Exception:
+                        rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                    pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                    self.samples.append((sm, rs, pw))
+                except Exception as e:  # pragma: no cover
+                    self.err = str(e)
+                self._stop.wait(self.period)
+
+        self.t = threading.Thread(target=run, daemon=True)
+        self.t.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        if self._stop is not None:
+            self._stop.set()
+            self.t.join(timeout=2)
 
     def summary(self):
-        if self.proc is None or not self.path:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"]}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({name for _, rs, _ in self.samples for bit, name in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_sm, "sm_min_mhz": min(sm),
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": max(x[2] for x in self.samples), "source": "nvml"}
 
 
 def _barrier(ws):
@@ -118,13 +138,22 @@ def _max_over_ranks(x: float, ws: int) -> float:
     return float(t.item())
 
 
-def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: int, e2e: bool):
+def pv_mode(w: W.Workload, choice: str) -> int:
+    """auto: the two-level scheme where the workload's recipe names it, else the
+    TMEM FP32 accumulator (tcgen05 accumulates FP8 products in full FP32)."""
+    if choice == "auto":
+        return 0 if w.names_two_level else 1
+    return {"two_level": 0, "tmem_fp32": 1}[choice]
+
+
+def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: int, e2e: bool,
+             pv_accum: int = 0, time_other_mode: bool = False):
     from quantized_attention_block_b200 import sage
 
     q, k, v = W.make_qkv(w, seed=w.seed + rank)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     p = sage.make_params(qd, kd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
-                         smooth_q=w.smooth_q, bq=w.bq, bk=w.bk)
+                         smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=pv_accum)
     wsp = sage.alloc_workspace(p)
     o = torch.empty_like(qd)
     stream = torch.cuda.current_stream()
@@ -159,6 +188,21 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
     ms_attn = _max_over_ranks(ms_attn, ws)
     res = {"ms_step": ms_step, "ms_attn": ms_attn, "ms_quant": ms_step - ms_attn, "clocks": clk.summary(),
            "gpu_launches": launches_per_step * steps}
+    if time_other_mode:
+        # kernel time of the other P~V accumulation mode on the same inputs (for the record)
+        p2 = sage.make_params(qd, kd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                              smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=1 - pv_accum)
+        view = sage.sage_quant_qkv(qd, kd, vd, p2, wsp, stream)
+        for _ in range(3):
+            sage.sage_attn_fwd_quantized(view, o, p2, stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(3, steps // 2)
+        e0.record(stream)
+        for _ in range(n):
+            sage.sage_attn_fwd_quantized(view, o, p2, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res["ms_attn_other_mode"] = _max_over_ranks(e0.elapsed_time(e1) / n, ws)
 
     if e2e:
         qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
@@ -169,7 +213,8 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
             sage.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
-                               smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, out=o, workspace=wsp, stream=stream)
+                               smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=pv_accum, out=o, workspace=wsp,
+                               stream=stream)
             oh.copy_(o, non_blocking=True)
 
         for _ in range(2):
@@ -222,19 +267,25 @@ def oracle_sample(w: W.Workload, heads: int, tiles: int, threads: int):
 
 
 def main():
+    faulthandler.enable()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sage", "reference"], default="sage")
     ap.add_argument("--workload", default="prefill")
     ap.add_argument("--extra-workloads", default="video,gqa")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--override", default="", help="workload fields, e.g. B=1,Hq=16,Hkv=16 (profiling cases)")
+    ap.add_argument("--pv-accum", choices=["auto", "two_level", "tmem_fp32"], default="auto")
     args = ap.parse_args()
 
     ws, rank, local = _dist()
     w = W.get(args.workload)
+    if args.override:
+        kv = dict(x.split("=") for x in args.override.split(","))
+        w = w.with_(name=w.name + "@" + args.override.replace(",", "_"), **{k: int(v) for k, v in kv.items()})
     metric = "quantized attn fwd TOPS on 1 B200 (N=4K-32K, d=64/128); % of tensor peak"
     threads = os.cpu_count() or 1
     config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
@@ -273,15 +324,21 @@ def main():
 
     peaks, peak_kind = _peaks()
     peak_tops = peaks["bf16_tflops_sustained"] * INT8_FP8_PER_BF16
-    res = run_sage(w, args.steps, args.warmup, ws, rank, local, not args.no_e2e)
+    mode = pv_mode(w, args.pv_accum)
+    config["pv_accum"] = ["two_level", "tmem_fp32"][mode]
+    res = run_sage(w, args.steps, args.warmup, ws, rank, local, not args.no_e2e, mode,
+                   time_other_mode=not args.no_e2e)
     ops = w.ops()
     value = ws * ops / (res["ms_step"] * 1e-3) / 1e12
     attn_tops = ops / (res["ms_attn"] * 1e-3) / 1e12
     extra = {}
     for name in [x for x in args.extra_workloads.split(",") if x and x != "none"]:
         we = W.get(name)
-        r = run_sage(we, max(3, args.steps // 4), 3, ws, rank, local, False)
-        extra[we.name] = {"step_tops": we.ops() / (r["ms_step"] * 1e-3) / 1e12,
+        me = pv_mode(we, args.pv_accum)
+        r = run_sage(we, max(3, args.steps // 4), 3, ws, rank, local, False, me, time_other_mode=True)
+        extra[we.name] = {"pv_accum": ["two_level", "tmem_fp32"][me],
+                          "step_tops": we.ops() / (r["ms_step"] * 1e-3) / 1e12,
+                          "attn_kernel_tops_other_mode": we.ops() / (r["ms_attn_other_mode"] * 1e-3) / 1e12,
                           "attn_kernel_tops": we.ops() / (r["ms_attn"] * 1e-3) / 1e12,
                           "ms_step": r["ms_step"], "ms_attn": r["ms_attn"],
                           "attn_frac_of_peak": we.ops() / (r["ms_attn"] * 1e-3) / 1e12 / peak_tops}
@@ -292,6 +349,8 @@ def main():
         "data": "synthetic (seeded, recipe of the workload)", "config": config,
         "kernel_only_tops": attn_tops,
         "per_kernel_ms": {"quant_total": res["ms_quant"], "attn_i8f8": res["ms_attn"]},
+        "attn_kernel_tops_other_pv_accum": (ops / (res["ms_attn_other_mode"] * 1e-3) / 1e12
+                                            if "ms_attn_other_mode" in res else None),
         "roofline": {"bound": "tensor", "kernel": "attn_i8f8_kernel", "achieved": attn_tops,
                      "peak": peak_tops, "unit": "TFLOP/s", "frac": attn_tops / peak_tops,
                      "peak_source": f"{peak_kind}: bf16 sustained {peaks['bf16_tflops_sustained']} x "

@@ -67,7 +67,17 @@ typedef struct {
     int32_t smooth_q;          /* 1: subtract each Q block's mean and add delta_S back */
     int32_t bq;                /* Q quantisation block in rows: 64 or 128 */
     int32_t bk;                /* K quantisation block in rows: 64 or 128 */
+    int32_t pv_accum;          /* FP32 accumulation of P~V across key tiles:
+                                  SAGE_PV_TWO_LEVEL (0): each tile's P^V lands in a
+                                    fresh TMEM tile, then O = e^(m_old-m) O + O_t on
+                                    CUDA cores (SageAttention2 Algorithm 1, level 2);
+                                  SAGE_PV_TMEM_FP32 (1): P^V accumulates in one FP32
+                                    TMEM accumulator, rescaled on CUDA cores only for
+                                    rows whose max grew (tcgen05 keeps full FP32 in
+                                    the accumulator: see sage_debug_f8_accum_probe) */
 } sage_params;
+
+enum { SAGE_PV_TWO_LEVEL = 0, SAGE_PV_TMEM_FP32 = 1 };
 
 /*
  * Device views of the quantised tensors produced by sage_quant_qkv (all
@@ -179,6 +189,18 @@ SAGE_API sage_status sage_debug_bounded_wait(uint32_t timeout_us, void *stream);
  */
 SAGE_API sage_status sage_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *o,
                                            const sage_params *p, void *stream);
+
+/*
+ * Accumulator-precision probe of the FP8 tensor-core path (tcgen05.mma
+ * kind::f8f6f4, FP32 accumulator).  The SageAttention2 note ("5. Numerical
+ * Considerations") reports that Ada/Hopper FP8 MMAs keep only ~13 mantissa
+ * bits in their accumulator, the reason for the two-level accumulation.
+ * Writes 8 floats to out8 (device) whose exact values are
+ *   1+2^-18, 1+2^-14, 1+2^-12, 256, 32, 4096+2^-10, 1+2^-18, 1+2^-13
+ * (cases 5-7 accumulate across two MMAs).  Comparing them with these values
+ * shows how many accumulator bits the hardware keeps.
+ */
+SAGE_API sage_status sage_debug_f8_accum_probe(float *out8, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 SAGE_API const char *sage_status_string(sage_status s);

@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -40,6 +41,7 @@ sage_status check_params(const sage_params* p, Dims* d) {
       (p->smooth_q != 0 && p->smooth_q != 1))
     return SAGE_ERR_INVALID_ARG;
   if (std::isnan(p->sm_scale) || std::isinf(p->sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (p->pv_accum != SAGE_PV_TWO_LEVEL && p->pv_accum != SAGE_PV_TMEM_FP32) return SAGE_ERR_INVALID_ARG;
   d->B = p->B;
   d->Hq = p->Hq;
   d->Hkv = p->Hkv;
@@ -149,6 +151,17 @@ sage_status make_maps(const sage_quant_view* v, const Dims& d, CUtensorMap* mQ, 
   return SAGE_OK;
 }
 
+// Scheduling of the two softmax warpgroups: taking turns (ping-pong) or running
+// concurrently.  SAGE_SOFTMAX_PINGPONG=0/1 overrides the per-mode default.
+int softmax_pingpong(int two_level) {
+  static const int env = [] {
+    const char* v = std::getenv("SAGE_SOFTMAX_PINGPONG");
+    return v ? std::atoi(v) : -1;
+  }();
+  (void)two_level;
+  return env >= 0 ? (env != 0) : 0;  // measured: concurrent is faster in both modes
+}
+
 AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d) {
   AttnArgs a{};
   a.B = (int)d.B;
@@ -170,10 +183,13 @@ AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d
   a.s_v = v->s_v;
   a.dS = p->smooth_q ? v->dS : nullptr;
   a.out_fp16 = p->dtype == SAGE_FP16;
+  a.two_level = p->pv_accum == SAGE_PV_TWO_LEVEL;
+  a.pingpong = softmax_pingpong(a.two_level);
   return a;
 }
 
 sage_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
+
 
 }  // namespace
 
@@ -225,7 +241,11 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
   a.dS = view->dS;
   a.ksum = reinterpret_cast<double*>(base + L.ksum);
   a.vamax = reinterpret_cast<unsigned*>(base + L.vamax);
-  return from_cuda(launch_quant(a, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
+  CUtensorMap mVt;
+  if (!map_2d_u8(&mVt, view->v8t, (uint64_t)d.Np, (uint64_t)(d.B * d.Hkv * d.D), kTile, (uint32_t)d.D,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return SAGE_ERR_CUDA;
+  return from_cuda(launch_quant(a, mVt, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status sage_attn_fwd_quantized(const sage_quant_view* view, void* o, const sage_params* p, void* stream) {
@@ -302,6 +322,13 @@ sage_status sage_debug_bounded_wait(uint32_t timeout_us, void* stream) {
       cudaSuccess)
     return SAGE_ERR_CUDA;
   return sage_last_device_error(stream);
+}
+
+sage_status sage_debug_f8_accum_probe(float* out8, void* stream) {
+  if (!out8 || !aligned16(out8)) return SAGE_ERR_INVALID_ARG;
+  sage_status s = check_arch();
+  if (s != SAGE_OK) return s;
+  return from_cuda(launch_f8_accum_probe(out8, static_cast<cudaStream_t>(stream)));
 }
 
 const char* sage_status_string(sage_status s) {

@@ -23,11 +23,17 @@
 //   WG1  softmax of Q tile 0    (thread = one Q row = one TMEM lane)
 //   WG2  softmax of Q tile 1
 //   WG3  level-2 accumulation O = alpha O + O_t for both tiles, and the epilogue
-// The two softmax warpgroups take turns (ping-pong on mbarriers), so the MMA
-// and correction chain of one tile runs while the other tile's softmax owns
-// the issue slots.  TMEM (512 columns): tile i's S_i / O_t_i share columns
-// [128 i, 128 i + 128) (P goes through shared memory, so S is dead once the
-// softmax has read it); O_i lives at [256 + D i, 256 + D (i + 1)).
+// The two softmax warpgroups run concurrently (two softmax warps per SM
+// sub-partition hide each other's latencies); an optional ping-pong mode makes
+// them take turns on mbarriers.  TMEM (512 columns): S_i at [128 i, 128 i + 128)
+// and O_i at [256 + D i, 256 + D (i + 1)).  P goes through shared memory.
+// Two P~V accumulation modes (template TWO_LEVEL):
+//   two-level: PV(i, j) writes a fresh O_t into S_i's columns (S is dead once
+//     the softmax read it); the correction warpgroup adds it into O_i on CUDA
+//     cores: O_i = alpha O_i + O_t (SageAttention2 Algorithm 1, level 2).
+//   TMEM accumulator: PV(i, j) accumulates into O_i itself (tcgen05 keeps the
+//     FP8 products' sum in full FP32); before it, the correction warpgroup
+//     rescales the rows of O_i whose max grew (alpha != 1; alpha == 1 is exact).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -43,7 +49,7 @@ constexpr int kThreadsAttn = 512;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 
 // per-warpgroup register budgets after setmaxnreg (sum x 128 <= 65536)
-constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 176, kRegsCorrection = 104;
+constexpr uint32_t kRegsProducer = 40, kRegsSoftmax = 192, kRegsCorrection = 88;
 static_assert(kRegsProducer + 2 * kRegsSoftmax + kRegsCorrection <= 512, "register split exceeds the launch");
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -60,7 +66,7 @@ struct Smem {
   static constexpr uint32_t oAlpha = oP + 2 * kP;        // float[2][128]
   static constexpr uint32_t oL = oAlpha + 2 * 128 * 4;   // float[2][128]
   static constexpr uint32_t oBar = oL + 2 * 128 * 4;
-  static constexpr uint32_t kNumBars = 1 + 3 * kStages + 6 * 2;
+  static constexpr uint32_t kNumBars = 1 + 3 * kStages + 7 * 2 + 1;
   static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = oTmem + 16 + 1024;  // + alignment slack
 };
@@ -86,12 +92,15 @@ struct Bars {
   uint64_t* s_full;    // [2]  QK^T of tile i done            (tcgen05.commit)
   uint64_t* p_full;    // [2]  P_i and alpha_i written         (128 softmax threads)
   uint64_t* ot_full;   // [2]  O_t of tile i done              (tcgen05.commit)
-  uint64_t* r_free;    // [2]  O_t_i consumed, columns free    (128 correction threads)
+  uint64_t* r_free;    // [2]  S_i columns free for the next QK^T (two-level: correction
+                       //      consumed O_t_i; TMEM accumulator: softmax read S_i)
   uint64_t* turn;      // [2]  softmax ping-pong: tile i may run (128 threads of the other tile)
   uint64_t* l_ready;   // [2]  final l of tile i in shared memory
+  uint64_t* o_ready;   // [2]  (TMEM accumulator mode) O_i rescaled for the next P V
+  uint64_t* mma_done;  // all tensor-core work of the CTA retired (one commit at the end)
 };
 
-template <int D, bool CAUSAL, bool HAS_DS, typename TO>
+template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -122,6 +131,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   bar.r_free = bar.ot_full + 2;
   bar.turn = bar.r_free + 2;
   bar.l_ready = bar.turn + 2;
+  bar.o_ready = bar.l_ready + 2;
+  bar.mma_done = bar.o_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oTmem);
 
   // ---- work: (b, h, pair of Q tiles), heavy causal pairs first
@@ -156,7 +167,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       mbar_init(&bar.r_free[i], 128);
       mbar_init(&bar.turn[i], 128);
       mbar_init(&bar.l_ready[i], 128);
+      mbar_init(&bar.o_ready[i], 128);
     }
+    mbar_init(bar.mma_done, 1);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -203,7 +216,6 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       if (lane == 0) {
         const uint32_t aP0 = smem_u32(sP);
         bool ok = mbar_wait(bar.q_full, 0);
-        uint32_t last_ot[2] = {0, 0}, last_s[2] = {0, 0};  // commits per tile
         auto issue_qk = [&](int i, int j) {
           const int s = j % kStages;
           const uint32_t aQ = smem_u32(sQ + i * L::kQ), aK = smem_u32(sK + s * L::kK);
@@ -212,51 +224,71 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             mma_i8(tmem + 128 * i, make_sdesc(aQ + kk * 32, kSboQK, kSwzQK), make_sdesc(aK + kk * 32, kSboQK, kSwzQK),
                    kIdescQK, kk > 0 ? 1u : 0u);
           mma_commit(&bar.s_full[i]);
-          ++last_s[i];
         };
         auto issue_pv = [&](int i, int j) {
           const int s = j % kStages;
           const uint32_t aP = aP0 + i * L::kP, aV = smem_u32(sV + s * L::kV);
+          // two-level: a fresh O_t tile in S_i's columns; else accumulate into O_i
+          const uint32_t dst = TWO_LEVEL ? tmem + 128 * i : tmem + 256 + D * i;
 #pragma unroll
           for (int kk = 0; kk < kTile / 32; ++kk)
-            mma_f8f6f4(tmem + 128 * i, make_sdesc(aP + kk * 32, 1024, kSwizzle128B),
-                       make_sdesc(aV + kk * 32, 1024, kSwizzle128B), kIdescPV, kk > 0 ? 1u : 0u);
+            mma_f8f6f4(dst, make_sdesc(aP + kk * 32, 1024, kSwizzle128B), make_sdesc(aV + kk * 32, 1024, kSwizzle128B),
+                       kIdescPV, (kk > 0 || (!TWO_LEVEL && j > 0)) ? 1u : 0u);
           mma_commit(&bar.ot_full[i]);
-          ++last_ot[i];
         };
-        if (ok) ok = mbar_wait(&bar.k_full[0], 0);
-        if (ok) {
-          tc_fence_after();
-          for (int i = 0; i < 2; ++i)
-            if (nTi[i] > 0) issue_qk(i, 0);
-        }
-        for (int j = 0; j < nT && ok; ++j) {
-          const int s = j % kStages;
-          if (!(ok = mbar_wait(&bar.v_full[s], (j / kStages) & 1))) break;
-          bool k_next = false;
-          for (int i = 0; i < 2 && ok; ++i) {
-            if (j < nTi[i]) {
-              if (!(ok = mbar_wait(&bar.p_full[i], j & 1))) break;
+        // Two independent per-tile chains, each op issued as soon as its inputs
+        // are ready (non-blocking polls), so one tile never holds the other back.
+        //   QK(i,j): K_j landed; j > 0: S_i columns free (r_free) and, two-level,
+        //            PV(i,j-1) issued (its O_t shares those columns)
+        //   PV(i,j): QK(i,j) issued; V_j landed; P_i(j) written; TMEM-accumulator
+        //            mode, j > 0: O_i rescaled (o_ready)
+        // Stage j of the K/V ring is released once every active tile issued PV(i,j).
+        int next_qk[2] = {0, 0}, next_pv[2] = {0, 0};
+        int released = 0;
+        uint64_t t_idle = 0;
+        while (ok) {
+          bool progress = false;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int jq = next_qk[i], jp = next_pv[i];
+            if (jq < nTi[i] && (!TWO_LEVEL || jp >= jq) &&
+                mbar_test_wait(smem_u32(&bar.k_full[jq % kStages]), (jq / kStages) & 1) &&
+                (jq == 0 || mbar_test_wait(smem_u32(&bar.r_free[i]), (jq - 1) & 1))) {
               tc_fence_after();
-              issue_pv(i, j);
+              issue_qk(i, jq);
+              next_qk[i] = jq + 1;
+              progress = true;
             }
-            if (j + 1 < nTi[i]) {
-              if (!k_next) {
-                if (!(ok = mbar_wait(&bar.k_full[(j + 1) % kStages], ((j + 1) / kStages) & 1))) break;
-                k_next = true;
-              }
-              if (!(ok = mbar_wait(&bar.r_free[i], j & 1))) break;
+            if (jp < nTi[i] && next_qk[i] > jp && mbar_test_wait(smem_u32(&bar.p_full[i]), jp & 1) &&
+                mbar_test_wait(smem_u32(&bar.v_full[jp % kStages]), (jp / kStages) & 1) &&
+                (TWO_LEVEL || jp == 0 || mbar_test_wait(smem_u32(&bar.o_ready[i]), (jp - 1) & 1))) {
               tc_fence_after();
-              issue_qk(i, j + 1);
+              issue_pv(i, jp);
+              next_pv[i] = jp + 1;
+              progress = true;
             }
           }
-          mma_commit(&bar.kv_empty[s]);
+          while (released < nT && (next_pv[0] > released || released >= nTi[0]) &&
+                 (next_pv[1] > released || released >= nTi[1])) {
+            mma_commit(&bar.kv_empty[released % kStages]);
+            ++released;
+          }
+          if (next_pv[0] >= nTi[0] && next_pv[1] >= nTi[1] && released >= nT) break;
+          if (progress) {
+            t_idle = 0;
+          } else if (t_idle == 0) {
+            __nanosleep(32);
+            t_idle = globaltimer_ns();
+          } else if (globaltimer_ns() - t_idle > g_wait_limit_ns) {
+            record_error(kDevErrTimeout);
+            ok = false;
+          } else {
+            __nanosleep(32);
+          }
         }
         // every tensor-core op retired before TMEM is released
-        for (int i = 0; i < 2; ++i) {
-          if (last_s[i] > 0) mbar_wait(&bar.s_full[i], (last_s[i] - 1) & 1);
-          if (last_ot[i] > 0) mbar_wait(&bar.ot_full[i], (last_ot[i] - 1) & 1);
-        }
+        mma_commit(bar.mma_done);
+        mbar_wait(bar.mma_done, 0);
       }
       __syncwarp();
     }
@@ -279,8 +311,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 
     for (int j = 0; j < nT && ok; ++j) {
       // ping-pong: tile 0 runs iteration j after tile 1 finished j-1; tile 1 after tile 0 finished j
-      if (ti == 0 && j > 0) ok = mbar_wait_warp(&bar.turn[0], (j - 1) & 1);
-      if (ti == 1) ok = ok && mbar_wait_warp(&bar.turn[1], j & 1);
+      if (a.pingpong && ti == 0 && j > 0) ok = mbar_wait_warp(&bar.turn[0], (j - 1) & 1);
+      if (a.pingpong && ti == 1) ok = ok && mbar_wait_warp(&bar.turn[1], j & 1);
       if (!ok) break;
       if (j < nTi[ti]) {
         if (!(ok = mbar_wait_warp(&bar.s_full[ti], j & 1))) break;
@@ -294,7 +326,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         const float a_lo = row_scale * __ldg(sk + min(col0 / a.bk, a.Tn - 1));
         const float a_hi = row_scale * __ldg(sk + min((col0 + 64) / a.bk, a.Tn - 1));
         tmem_ld_wait();
-        // S region is now free for O_t (the MMA overwrites it after p_full)
+        if (!TWO_LEVEL) {  // S_i is in registers: the next QK^T may overwrite its columns
+          tc_fence_before();
+          mbar_arrive(&bar.r_free[ti]);
+        }
         // t = float(acc) * a (+ delta_S * sm_scale * log2 e), in place (as float bits)
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
@@ -319,14 +354,27 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             if (col >= a.N || (CAUSAL && col > qrow)) s[c] = __float_as_uint(-INFINITY);
           }
         }
-        float mx = -INFINITY;
+        // row max: 8 independent 3-input chains, then a short tree (max is exact)
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) mx = fmax3(mx, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx8[k] = fmax3(mx8[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_new = fmaxf(m, mx);
         const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
         const float mm = (m_new == -INFINITY) ? 0.0f : m_new - kLog2_448;
+        // TMEM-accumulator mode: PV(j-1) must have read P_i before it is rewritten
+        // (two-level: guaranteed by the chain O_t -> correction -> next QK^T)
+        if (!TWO_LEVEL && j > 0 && !(ok = mbar_wait_warp(&bar.ot_full[ti], (j - 1) & 1))) break;
         // P = exp2(t - m + log2 448) -> E4M3 -> shared memory (128B-swizzled K-major)
-        float2 rs2 = make_float2(0.0f, 0.0f);
+        // row sum: 8 independent f32x2 partial sums (fp32 rounding order only)
+        float2 rs[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) rs[k] = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int grp = 0; grp < 8; ++grp) {
           uint32_t w[4];
@@ -339,11 +387,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                     make_float2(-mm, -mm));
             const float2 p0 = make_float2(ex2_approx(u0.x), ex2_approx(u0.y));
             const float2 p1 = make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
-            rs2 = fadd2(rs2, fadd2(p0, p1));
+            rs[e / 2] = fadd2(rs[e / 2], p0);
+            rs[e / 2 + 1] = fadd2(rs[e / 2 + 1], p1);
             w[e / 4] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
           }
           *reinterpret_cast<uint4*>(myP + ((grp ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        const float2 rs2 = fadd2(fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3])),
+                                 fadd2(fadd2(rs[4], rs[5]), fadd2(rs[6], rs[7])));
         s_alpha[ti * 128 + row] = alpha;
         tc_fence_before();
         fence_proxy_async_smem();
@@ -351,7 +402,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         l = fmaf(l, alpha, rs2.x + rs2.y);
         m = m_new;
       }
-      mbar_arrive(&bar.turn[ti ^ 1]);
+      if (a.pingpong) mbar_arrive(&bar.turn[ti ^ 1]);
     }
     s_l[ti * 128 + row] = l;
     mbar_arrive(&bar.l_ready[ti]);
@@ -363,40 +414,100 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
     uint32_t x[32], y[32];
-    for (int j = 0; j < nT && ok; ++j) {
-      for (int i = 0; i < 2; ++i) {
-        if (j >= nTi[i]) continue;
-        if (!(ok = mbar_wait_warp(&bar.ot_full[i], j & 1))) break;
-        if (!(ok = mbar_wait_warp(&bar.p_full[i], j & 1))) break;
-        tc_fence_after();
-        const float alpha = s_alpha[i * 128 + row];
-        const uint32_t tOt = tmem + 128 * i + lane_off, tO = tmem + 256 + D * i + lane_off;
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          tmem_ld32(tOt + c, x);
-          if (j > 0) tmem_ld32(tO + c, y);
-          tmem_ld_wait();
-          if (j > 0) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float2 o = ffma2(make_float2(__uint_as_float(y[e]), __uint_as_float(y[e + 1])),
-                                     make_float2(alpha, alpha),
-                                     make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])));
-              x[e] = __float_as_uint(o.x);
-              x[e + 1] = __float_as_uint(o.y);
+    if constexpr (TWO_LEVEL) {
+      for (int j = 0; j < nT && ok; ++j) {
+        for (int i = 0; i < 2; ++i) {
+          if (j >= nTi[i]) continue;
+          if (!(ok = mbar_wait_warp(&bar.ot_full[i], j & 1))) break;
+          if (!(ok = mbar_wait_warp(&bar.p_full[i], j & 1))) break;
+          tc_fence_after();
+          const float alpha = s_alpha[i * 128 + row];
+          const uint32_t tOt = tmem + 128 * i + lane_off, tO = tmem + 256 + D * i + lane_off;
+          if (j == 0) {
+  #pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              tmem_ld32(tOt + c, x);
+              tmem_ld_wait();
+              tmem_st32(tO + c, x);
+            }
+          } else {
+            // O = alpha * O + O_t in 16-column chunks; the loads of chunk c + 1
+            // are in flight while chunk c is combined and stored.
+            uint32_t* xa = x;
+            uint32_t* ya = y;
+            uint32_t* xb = x + 16;
+            uint32_t* yb = y + 16;
+            tmem_ld16p(tOt, xa);
+            tmem_ld16p(tO, ya);
+            tmem_ld_wait();
+  #pragma unroll
+            for (int c = 0; c < D; c += 16) {
+              uint32_t* xc = (c / 16) % 2 == 0 ? xa : xb;
+              uint32_t* yc = (c / 16) % 2 == 0 ? ya : yb;
+              uint32_t* xn = (c / 16) % 2 == 0 ? xb : xa;
+              uint32_t* yn = (c / 16) % 2 == 0 ? yb : ya;
+              if (c + 16 < D) {
+                tmem_ld16p(tOt + c + 16, xn);
+                tmem_ld16p(tO + c + 16, yn);
+              }
+  #pragma unroll
+              for (int e = 0; e < 16; e += 2) {
+                const float2 o = ffma2(make_float2(__uint_as_float(yc[e]), __uint_as_float(yc[e + 1])),
+                                       make_float2(alpha, alpha),
+                                       make_float2(__uint_as_float(xc[e]), __uint_as_float(xc[e + 1])));
+                xc[e] = __float_as_uint(o.x);
+                xc[e + 1] = __float_as_uint(o.y);
+              }
+              tmem_st16p(tO + c, xc);
+              if (c + 16 < D) tmem_ld_wait();
             }
           }
-          tmem_st32(tO + c, x);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&bar.r_free[i]);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bar.r_free[i]);
+      }
+    } else {
+      // O_i accumulates in TMEM; before PV(i, j) adds tile j, rows whose max grew
+      // are rescaled by alpha = e^(m_old - m_new).  A warp whose 32 rows all have
+      // alpha == 1 leaves O_i untouched (exact).
+      // (every phase of p_full is waited in order, j = 0 included: a parity wait
+      // on a phase two ahead of the barrier would pass at once)
+      for (int j = 0; j < nT && ok; ++j) {
+        for (int i = 0; i < 2; ++i) {
+          if (j >= nTi[i]) continue;
+          if (!(ok = mbar_wait_warp(&bar.p_full[i], j & 1))) break;
+          if (j == 0) continue;
+          if (!(ok = mbar_wait_warp(&bar.ot_full[i], (j - 1) & 1))) break;
+          tc_fence_after();
+          const float alpha = s_alpha[i * 128 + row];
+          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+            const uint32_t tO = tmem + 256 + D * i + lane_off;
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              tmem_ld32(tO + c, x);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float2 o = fmul2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])),
+                                       make_float2(alpha, alpha));
+                x[e] = __float_as_uint(o.x);
+                x[e + 1] = __float_as_uint(o.y);
+              }
+              tmem_st32(tO + c, x);
+            }
+            tmem_st_wait();
+          }
+          tc_fence_before();
+          mbar_arrive(&bar.o_ready[i]);
+        }
       }
     }
     // epilogue: out = O / l * delta_V   (l carries the 448)
     for (int i = 0; i < 2 && ok; ++i) {
       if (nTi[i] == 0) continue;
       if (!(ok = mbar_wait_warp(&bar.l_ready[i], 0))) break;
+      if (!TWO_LEVEL && !(ok = mbar_wait_warp(&bar.ot_full[i], (nTi[i] - 1) & 1))) break;
       tc_fence_after();
       const float inv_l = 1.0f / s_l[i * 128 + row];
       const int64_t qrow = (int64_t)(2 * pr + i) * kTile + row;
@@ -500,6 +611,96 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// Accumulator-precision probe of tcgen05.mma kind::f8f6f4 (M=128, N=128).
+// Case r uses A row r and B row r, so D[r][r] = sum_k A[r][k] B[r][k]; the two
+// MMAs read K bytes [0, 32) then [32, 64) (accumulating), so cases 5-7 test
+// the carry of the FP32 accumulator across instructions.  Operands are E4M3:
+//   0: [1, 2^-9].[1, 2^-9]            = 1 + 2^-18      (18 bits)
+//   1: [1, 2^-8].[1, 2^-6]            = 1 + 2^-14
+//   2: [1, 2^-6].[1, 2^-6]            = 1 + 2^-12
+//   3: [256, 2^-9].[1, 2^-9]          = 256 + 2^-18    (below fp32 ulp: 256)
+//   4: 32 x [1].[1]                   = 32
+//   5: [64].[64]  then [2^-5].[2^-5]  = 4096 + 2^-10   (22 bits, across MMAs)
+//   6: [1].[1]    then [2^-9].[2^-9]  = 1 + 2^-18      (across MMAs)
+//   7: [1].[1]    then 32 x 2^-9.2^-9 = 1 + 2^-13      (across MMAs)
+// out[r] = D[r][r] for r < 8.
+__global__ void __launch_bounds__(128, 1) f8_accum_probe_kernel(float* out) {
+  constexpr uint32_t kIdesc = make_idesc(/*F32*/ 1, /*E4M3*/ 0, /*E4M3*/ 0, 128, 128);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + 16384;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 32768);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  const int r = threadIdx.x, warp = r / 32, lane = r % 32;
+  uint8_t a[64], bb[64];
+#pragma unroll
+  for (int k = 0; k < 64; ++k) { a[k] = 0; bb[k] = 0; }
+  const uint8_t one = 0x38, m9 = 0x01, m8 = 0x02, m6 = 0x08, c64 = 0x68, m5 = 0x10, c256 = 0x78;
+  switch (r) {
+    case 0: a[0] = one; a[1] = m9; bb[0] = one; bb[1] = m9; break;
+    case 1: a[0] = one; a[1] = m8; bb[0] = one; bb[1] = m6; break;
+    case 2: a[0] = one; a[1] = m6; bb[0] = one; bb[1] = m6; break;
+    case 3: a[0] = c256; a[1] = m9; bb[0] = one; bb[1] = m9; break;
+    case 4: for (int k = 0; k < 32; ++k) { a[k] = one; bb[k] = one; } break;
+    case 5: a[0] = c64; bb[0] = c64; a[32] = m5; bb[32] = m5; break;
+    case 6: a[0] = one; bb[0] = one; a[32] = m9; bb[32] = m9; break;
+    case 7: a[0] = one; bb[0] = one; for (int k = 32; k < 64; ++k) { a[k] = m9; bb[k] = m9; } break;
+    default: break;
+  }
+  // row r of a 128-byte-swizzled K-major tile: 16-byte chunk c at (c ^ (r & 7))
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t wa[4] = {0, 0, 0, 0}, wb[4] = {0, 0, 0, 0};
+    if (c < 4) {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        wa[u / 4] |= (uint32_t)a[c * 16 + u] << (8 * (u % 4));
+        wb[u / 4] |= (uint32_t)bb[c * 16 + u] << (8 * (u % 4));
+      }
+    }
+    *reinterpret_cast<uint4*>(sA + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    *reinterpret_cast<uint4*>(sB + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+  }
+  fence_proxy_async_smem();
+  if (r == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (r == 0) {
+    const uint32_t aA = smem_u32(sA), aB = smem_u32(sB);
+    mma_f8f6f4(tmem, make_sdesc(aA, 1024, kSwizzle128B), make_sdesc(aB, 1024, kSwizzle128B), kIdesc, 0u);
+    mma_f8f6f4(tmem, make_sdesc(aA + 32, 1024, kSwizzle128B), make_sdesc(aB + 32, 1024, kSwizzle128B), kIdesc, 1u);
+    mma_commit(bar);
+  }
+  __syncwarp();
+  if (mbar_wait_warp(bar, 0)) {
+    tc_fence_after();
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), v);
+    tmem_ld_wait();
+    if (warp == 0 && lane < 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u == lane) out[lane] = __uint_as_float(v[u]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // A wait nobody ends: the bounded wait gives up, records the timeout, returns.
 __global__ void bounded_wait_probe_kernel() {
   __shared__ uint64_t bar;
@@ -512,10 +713,10 @@ __global__ void bounded_wait_probe_kernel() {
   __syncthreads();
 }
 
-template <int D, bool CAUSAL, bool HAS_DS, typename TO>
+template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO>
 cudaError_t launch_attn_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                           cudaStream_t st) {
-  auto kern = attn_i8f8_kernel<D, CAUSAL, HAS_DS, TO>;
+  auto kern = attn_i8f8_kernel<D, CAUSAL, HAS_DS, TWO_LEVEL, TO>;
   const int smem = (int)Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -525,15 +726,21 @@ cudaError_t launch_attn_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUten
   return cudaGetLastError();
 }
 
+template <int D, bool CAUSAL, bool TWO_LEVEL>
+cudaError_t launch_attn_m(const AttnArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                          cudaStream_t st) {
+  if (a.dS) {
+    return a.out_fp16 ? launch_attn_t<D, CAUSAL, true, TWO_LEVEL, __half>(a, q, k, v, st)
+                      : launch_attn_t<D, CAUSAL, true, TWO_LEVEL, __nv_bfloat16>(a, q, k, v, st);
+  }
+  return a.out_fp16 ? launch_attn_t<D, CAUSAL, false, TWO_LEVEL, __half>(a, q, k, v, st)
+                    : launch_attn_t<D, CAUSAL, false, TWO_LEVEL, __nv_bfloat16>(a, q, k, v, st);
+}
+
 template <int D, bool CAUSAL>
 cudaError_t launch_attn_d(const AttnArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                           cudaStream_t st) {
-  if (a.dS) {
-    return a.out_fp16 ? launch_attn_t<D, CAUSAL, true, __half>(a, q, k, v, st)
-                      : launch_attn_t<D, CAUSAL, true, __nv_bfloat16>(a, q, k, v, st);
-  }
-  return a.out_fp16 ? launch_attn_t<D, CAUSAL, false, __half>(a, q, k, v, st)
-                    : launch_attn_t<D, CAUSAL, false, __nv_bfloat16>(a, q, k, v, st);
+  return a.two_level ? launch_attn_m<D, CAUSAL, true>(a, q, k, v, st) : launch_attn_m<D, CAUSAL, false>(a, q, k, v, st);
 }
 
 }  // namespace
@@ -557,6 +764,14 @@ cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUt
     if (e != cudaSuccess) return e;
     qk_probe_kernel<64><<<1, 128, smem, st>>>(tmQ, tmK, a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f8_accum_probe(float* out, cudaStream_t st) {
+  const int smem = 32768 + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(f8_accum_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  f8_accum_probe_kernel<<<1, 128, smem, st>>>(out);
   return cudaGetLastError();
 }
 

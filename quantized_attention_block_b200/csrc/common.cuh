@@ -44,16 +44,19 @@ struct AttnArgs {
   const float* dS;  // nullptr when smooth_q is off
   void* o;          // [B,Hq,N,D] bf16/fp16
   int out_fp16;
+  int two_level;  // 1: fresh O_t per key tile + FP32 add on CUDA cores; 0: TMEM FP32 accumulator
+  int pingpong;   // 1: the two softmax warpgroups take turns; 0: they run concurrently
   // probe mode (sage_debug_qk_int32)
   int probe_b, probe_h, probe_qtile, probe_ktile;
   int32_t* probe_out;
 };
 
 // launchers (defined in the .cu files)
-cudaError_t launch_quant(const QuantArgs& a, int is_fp16, cudaStream_t st);
+cudaError_t launch_quant(const QuantArgs& a, const CUtensorMap& tmVt, int is_fp16, cudaStream_t st);
 cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, cudaStream_t st);
 cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(cudaStream_t st);
+cudaError_t launch_f8_accum_probe(float* out, cudaStream_t st);
 
 }  // namespace sage

@@ -52,6 +52,9 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float (&x)[8]) {
   }
 }
 
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_float(__half x) { return __half2float(x); }
+
 // rows of a [r0, r0 + rows) block that lie below N
 __device__ __forceinline__ int rows_valid(int N, int64_t r0, int rows) {
   const int64_t v = (int64_t)N - r0;
@@ -134,13 +137,28 @@ __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
 // ---------------------------------------------------------------------------
 // Pass 2a: K (bk-row INT8 blocks of gamma(K)) and V (per-channel E4M3,
 // transposed to [d, Np]) for one 128-token tile.  grid (Np/128, B*Hkv)
+// V is staged in shared memory, each thread encodes 16-token runs of one
+// channel into a 128-byte-swizzled [d x 128] tile, and one TMA store writes
+// the tile to v8t (the same layout the attention kernel's TMA loads read).
+template <typename T, int D>
+struct KvSmem {
+  static constexpr int kPitch = D + 8;                          // padded V row (elements)
+  static constexpr uint32_t oVt = 0;                            // [D][128] bytes, 1024-aligned
+  static constexpr uint32_t oV = D * kTile;                     // [128][kPitch] T
+  static constexpr uint32_t kBytes = oV + kTile * kPitch * sizeof(T) + 1024;
+};
+
 template <typename T, int D, int BK>
-__global__ void __launch_bounds__(kThreads) kv_quant_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(kThreads) kv_quant_kernel(const __grid_constant__ CUtensorMap tmVt, QuantArgs a) {
   constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, PPB = BK / RG;  // passes per K block
   constexpr int NKB = kTile / BK;
+  using SL = KvSmem<T, D>;
+  extern __shared__ uint8_t kv_smem_raw[];
+  uint8_t* kv_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(kv_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sVt = kv_smem + SL::oVt;
+  T* sV = reinterpret_cast<T*>(kv_smem + SL::oV);
   __shared__ float s_km[D], s_sv[D], s_red[kThreads / 32];
   __shared__ float s_bmax[NKB];
-  __shared__ __align__(16) uint8_t s_vt[D][kTile + 16];
   const int bg = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
   const int valid = rows_valid(a.N, r0, kTile);
@@ -158,10 +176,19 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(QuantArgs a) {
     }
   }
   if (threadIdx.x < NKB) s_bmax[threadIdx.x] = 0.0f;
-  __syncthreads();
 
   const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
   const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)bg * a.N * D;
+
+  // ---- V tile -> shared memory (16-byte vectors; rows past N are zero)
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (r < valid) u = __ldg(reinterpret_cast<const uint4*>(V + (r0 + r) * D + ch * 8));
+    *reinterpret_cast<uint4*>(sV + r * SL::kPitch + ch * 8) = u;
+  }
+  __syncthreads();
 
   // ---- K: gamma(K) = K - km, per-block amax, INT8 codes
   float x[NP][8];
@@ -206,33 +233,34 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(QuantArgs a) {
     *reinterpret_cast<uint2*>(k8 + (r0 + r) * D + ch * 8) = pack8_i8(c8);
   }
 
-  // ---- V: E4M3(V / s_v[c]), transposed through shared memory
+  // ---- V: E4M3(V / s_v[c]) for 16-token runs of channel c, swizzled [D][128] tile
+  {
+    constexpr int TG = kThreads / D;           // token groups
+    constexpr int RUNS = kTile / 16 / TG;      // 16-token runs per thread
+    const int c = threadIdx.x % D, tg = threadIdx.x / D;
+    const float sv = s_sv[c];
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
-    float v[8];
-    if (r < valid) {
-      load8<T>(V + (r0 + r) * D + ch * 8, v);
-    } else {
+    for (int q = 0; q < RUNS; ++q) {
+      const int run = tg * RUNS + q;
+      uint32_t w[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.0f;
-    }
+      for (int u = 0; u < 16; u += 4) {
+        float f[4];
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const float sv0 = s_sv[ch * 8 + e], sv1 = s_sv[ch * 8 + e + 1];
-      const float f0 = (sv0 == 0.0f) ? 0.0f : __fdiv_rn(v[e], sv0);
-      const float f1 = (sv1 == 0.0f) ? 0.0f : __fdiv_rn(v[e + 1], sv1);
-      const uint32_t two = cvt_e4m3x2(f0, f1);
-      s_vt[ch * 8 + e][r] = (uint8_t)(two & 0xFF);
-      s_vt[ch * 8 + e + 1][r] = (uint8_t)(two >> 8);
+        for (int e = 0; e < 4; ++e) {
+          const float v = to_float(sV[(run * 16 + u + e) * SL::kPitch + c]);
+          f[e] = (sv == 0.0f) ? 0.0f : __fdiv_rn(v, sv);
+        }
+        w[u / 4] = cvt_e4m3x2(f[0], f[1]) | (cvt_e4m3x2(f[2], f[3]) << 16);
+      }
+      *reinterpret_cast<uint4*>(sVt + c * kTile + ((run ^ (c & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
+  fence_proxy_async_smem();
   __syncthreads();
-  uint8_t* vt = a.v8t + (int64_t)bg * D * a.Np + r0;
-  for (int i = threadIdx.x; i < D * (kTile / 16); i += kThreads) {
-    const int c = i / (kTile / 16), part = i % (kTile / 16);
-    *reinterpret_cast<uint4*>(vt + (int64_t)c * a.Np + part * 16) =
-        *reinterpret_cast<const uint4*>(&s_vt[c][part * 16]);
+  if (threadIdx.x == 0) {
+    tma_store_2d(&tmVt, sVt, (int)r0, bg * D);
+    tma_store_commit_and_wait_read();
   }
 }
 
@@ -365,7 +393,7 @@ __global__ void __launch_bounds__(kThreads) delta_s_kernel(QuantArgs a) {
 }
 
 template <typename T, int D>
-cudaError_t launch_quant_t(const QuantArgs& a, cudaStream_t st) {
+cudaError_t launch_quant_t(const QuantArgs& a, const CUtensorMap& tmVt, cudaStream_t st) {
   cudaError_t e;
   const int BHkv = a.B * a.Hkv, BHq = a.B * a.Hq;
   const int kv_tiles = (int)(a.Np / kTile);
@@ -376,10 +404,13 @@ cudaError_t launch_quant_t(const QuantArgs& a, cudaStream_t st) {
   e = cudaMemsetAsync(a.vamax, 0, sizeof(unsigned) * (size_t)BHkv * D, st);
   if (e != cudaSuccess) return e;
   kv_stats_kernel<T, D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(a);
-  if (a.bk == 64)
-    kv_quant_kernel<T, D, 64><<<dim3(kv_tiles, BHkv), kThreads, 0, st>>>(a);
-  else
-    kv_quant_kernel<T, D, 128><<<dim3(kv_tiles, BHkv), kThreads, 0, st>>>(a);
+  {
+    const int smem = (int)KvSmem<T, D>::kBytes;
+    auto kq = a.bk == 64 ? kv_quant_kernel<T, D, 64> : kv_quant_kernel<T, D, 128>;
+    e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kq<<<dim3(kv_tiles, BHkv), kThreads, smem, st>>>(tmVt, a);
+  }
   if (a.bq == 64)
     q_quant_kernel<T, D, 64><<<dim3((int)(a.Np / 64), BHq), kThreads, 0, st>>>(a);
   else
@@ -395,9 +426,11 @@ cudaError_t launch_quant_t(const QuantArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_quant(const QuantArgs& a, int is_fp16, cudaStream_t st) {
-  if (is_fp16) return a.D == 128 ? launch_quant_t<__half, 128>(a, st) : launch_quant_t<__half, 64>(a, st);
-  return a.D == 128 ? launch_quant_t<__nv_bfloat16, 128>(a, st) : launch_quant_t<__nv_bfloat16, 64>(a, st);
+cudaError_t launch_quant(const QuantArgs& a, const CUtensorMap& tmVt, int is_fp16, cudaStream_t st) {
+  if (is_fp16)
+    return a.D == 128 ? launch_quant_t<__half, 128>(a, tmVt, st) : launch_quant_t<__half, 64>(a, tmVt, st);
+  return a.D == 128 ? launch_quant_t<__nv_bfloat16, 128>(a, tmVt, st)
+                    : launch_quant_t<__nv_bfloat16, 64>(a, tmVt, st);
 }
 
 }  // namespace sage

@@ -25,7 +25,7 @@ STATUS_NAMES = {
 }
 EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd",
             "sage_debug_qk_int32", "sage_last_device_error", "sage_debug_bounded_wait",
-            "sage_status_string", "sage_attn_fwd_noalloc")
+            "sage_status_string", "sage_attn_fwd_noalloc", "sage_debug_f8_accum_probe")
 
 
 class SageError(RuntimeError):
@@ -38,7 +38,11 @@ class SageParams(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("sm_scale", ctypes.c_float), ("smooth_k", ctypes.c_int32),
-                ("smooth_q", ctypes.c_int32), ("bq", ctypes.c_int32), ("bk", ctypes.c_int32)]
+                ("smooth_q", ctypes.c_int32), ("bq", ctypes.c_int32), ("bk", ctypes.c_int32),
+                ("pv_accum", ctypes.c_int32)]
+
+
+PV_TWO_LEVEL, PV_TMEM_FP32 = 0, 1
 
 
 class SageQuantView(ctypes.Structure):
@@ -69,6 +73,7 @@ def lib() -> ctypes.CDLL:
         L.sage_debug_bounded_wait.argtypes = [ctypes.c_uint32, vp]
         L.sage_status_string.argtypes, L.sage_status_string.restype = [ctypes.c_int], ctypes.c_char_p
         L.sage_attn_fwd_noalloc.argtypes, L.sage_attn_fwd_noalloc.restype = [vp, vp, vp, vp, P, vp], ctypes.c_int
+        L.sage_debug_f8_accum_probe.argtypes, L.sage_debug_f8_accum_probe.restype = [vp, vp], ctypes.c_int
         for n in ("sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd", "sage_debug_qk_int32",
                   "sage_last_device_error", "sage_debug_bounded_wait"):
             getattr(L, n).restype = ctypes.c_int
@@ -87,12 +92,13 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> int:
 
 
 def make_params(q: torch.Tensor, k: torch.Tensor, *, causal: bool = False, sm_scale: Optional[float] = None,
-                smooth_k: bool = True, smooth_q: bool = False, bq: int = 128, bk: int = 64) -> SageParams:
+                smooth_k: bool = True, smooth_q: bool = False, bq: int = 128, bk: int = 64,
+                pv_accum: int = PV_TWO_LEVEL) -> SageParams:
     """Parameters for HND tensors q [B, Hq, N, d], k [B, Hkv, N, d]."""
     B, Hq, N, d = q.shape
     dt = {torch.bfloat16: 0, torch.float16: 1}.get(q.dtype, -1)
     return SageParams(B, Hq, k.shape[1], N, d, dt, int(causal), float(sm_scale if sm_scale else 0.0),
-                      int(smooth_k), int(smooth_q), bq, bk)
+                      int(smooth_k), int(smooth_q), bq, bk, int(pv_accum))
 
 
 def workspace_bytes(p: SageParams) -> int:
@@ -124,10 +130,12 @@ def sage_attn_fwd_quantized(view: SageQuantView, o: torch.Tensor, p: SageParams,
 
 
 def sage_attn_fwd(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = None, smooth_k: bool = True,
-                  smooth_q: bool = False, bq: int = 128, bk: int = 64, out: Optional[torch.Tensor] = None,
-                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                  smooth_q: bool = False, bq: int = 128, bk: int = 64, pv_accum: int = PV_TWO_LEVEL,
+                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
     """SageAttention forward: [B,Hq,N,d] x [B,Hkv,N,d] -> [B,Hq,N,d] (input dtype)."""
-    p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq, bk=bk)
+    p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq, bk=bk,
+                    pv_accum=pv_accum)
     if workspace is None:
         workspace = alloc_workspace(p, q.device)
     if out is None:
@@ -151,6 +159,17 @@ def sage_last_device_error(stream=None) -> int:
 
 def sage_debug_bounded_wait(timeout_us: int, stream=None) -> int:
     return int(lib().sage_debug_bounded_wait(int(timeout_us), _stream(stream)))
+
+
+F8_ACCUM_PROBE_EXACT = (1 + 2.0 ** -18, 1 + 2.0 ** -14, 1 + 2.0 ** -12, 256.0, 32.0, 4096 + 2.0 ** -10,
+                        1 + 2.0 ** -18, 1 + 2.0 ** -13)
+
+
+def sage_debug_f8_accum_probe(stream=None) -> torch.Tensor:
+    """The 8 probe sums of the FP8 tensor-core accumulator (exact values in F8_ACCUM_PROBE_EXACT)."""
+    out = torch.zeros(8, dtype=torch.float32, device="cuda")
+    _check(lib().sage_debug_f8_accum_probe(_ptr(out), _stream(stream)), "sage_debug_f8_accum_probe")
+    return out
 
 
 def view_tensors(view: SageQuantView, p: SageParams, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:

@@ -47,6 +47,8 @@ class Workload:
     qk_shared_bias_std: float = 0.0
     k_outlier_channels: int = 0
     k_outlier_mult: float = 1.0
+    # the recipe names the two-level FP32 accumulation of P~V explicitly
+    names_two_level: bool = False
 
     @property
     def sm_scale(self) -> float:
@@ -81,7 +83,7 @@ WORKLOADS: Dict[str, Workload] = {
     "long_gqa_causal_B1_Hq32_Hkv8_N32768_d128": Workload(
         "long_gqa_causal_B1_Hq32_Hkv8_N32768_d128", B=1, Hq=32, Hkv=8, N=32768, d=128,
         dtype=torch.bfloat16, causal=True, smooth_k=True, smooth_q=False, bq=128, bk=64,
-        nvfp4=False, seed=4, k_bias_std=3.0),
+        nvfp4=False, seed=4, k_bias_std=3.0, names_two_level=True),
     # NVFP4 (SageAttention3-style), non-causal, Q/K mean-smoothed.
     "nvfp4_B2_H24_N8192_d128": Workload(
         "nvfp4_B2_H24_N8192_d128", B=2, Hq=24, Hkv=24, N=8192, d=128,

@@ -19,9 +19,9 @@ def to_gpu(*ts):
     return [t.cuda() for t in ts]
 
 
-def gpu_quant(w: W.Workload, q, k, v):
+def gpu_quant(w: W.Workload, q, k, v, pv_accum: int = sage.PV_TWO_LEVEL):
     p = sage.make_params(q, k, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
-                         smooth_q=w.smooth_q, bq=w.bq, bk=w.bk)
+                         smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=pv_accum)
     ws = sage.alloc_workspace(p)
     qd, kd, vd = to_gpu(q, k, v)
     view = sage.sage_quant_qkv(qd, kd, vd, p, ws)
@@ -29,8 +29,8 @@ def gpu_quant(w: W.Workload, q, k, v):
     return p, ws, view, (qd, kd, vd)
 
 
-def gpu_attention(w: W.Workload, q, k, v):
-    p, ws, view, (qd, kd, vd) = gpu_quant(w, q, k, v)
+def gpu_attention(w: W.Workload, q, k, v, pv_accum: int = sage.PV_TWO_LEVEL):
+    p, ws, view, (qd, kd, vd) = gpu_quant(w, q, k, v, pv_accum)
     o = torch.empty_like(qd)
     sage.sage_attn_fwd_quantized(view, o, p)
     torch.cuda.synchronize()

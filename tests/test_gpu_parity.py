@@ -60,16 +60,30 @@ def test_qk_int32_tiles_bit_exact(name):
         np.testing.assert_array_equal(got, ref.astype(np.int32))
 
 
+PV_MODES = {"two_level": sage.PV_TWO_LEVEL, "tmem_fp32": sage.PV_TMEM_FP32}
+
+
+@pytest.mark.parametrize("mode", list(PV_MODES))
 @pytest.mark.parametrize("name", list(SMALL) + list(EDGE))
-def test_attention_matches_oracle_elementwise(name):
+def test_attention_matches_oracle_elementwise(name, mode):
     w = {**SMALL, **EDGE}[name]
     q, k, v = W.make_qkv(w)
-    p, ws, view, o = gpu_attention(w, q, k, v)
+    p, ws, view, o = gpu_attention(w, q, k, v, PV_MODES[mode])
     quant = oracle_quant(w, q, k, v)
     out = o.float().cpu().numpy()
     refs = np.stack([np.stack([oracle_rows(w, quant, b, h, 0, w.N) for h in range(w.Hq)]) for b in range(w.B)])
     m, ok = compare_out(refs, out)
     assert ok, m
+
+
+def test_pv_accumulation_modes_agree_closely():
+    """The TMEM FP32 accumulator and the two-level scheme differ only in FP32
+    rounding order (the accumulator keeps full FP32: see the probe test)."""
+    w = SMALL["gqa"]
+    q, k, v = W.make_qkv(w)
+    o0 = gpu_attention(w, q, k, v, sage.PV_TWO_LEVEL)[3].float()
+    o1 = gpu_attention(w, q, k, v, sage.PV_TMEM_FP32)[3].float()
+    assert (o0 - o1).abs().max().item() <= 1e-2
 
 
 def test_sage_attn_fwd_one_call_equals_two_step():
@@ -94,7 +108,7 @@ def test_bounded_wait_times_out_and_context_survives():
     gpu_attention(w, q, k, v)
 
 
-def test_rejects_non_sm100_inputs_cleanly():
+def test_rejects_invalid_arguments():
     w = SMALL["tiny"]
     q, k, v = W.make_qkv(w)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -115,14 +129,15 @@ def _sample_tiles(n_tiles, rng, k=3):
     return sorted(picks)
 
 
+@pytest.mark.parametrize("mode", list(PV_MODES))
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_quant_bit_exact_and_sampled_attention(name):
+def test_full_size_quant_bit_exact_and_sampled_attention(name, mode):
     """At the benchmark's sizes and launch configuration: every quantised value
     checked bit-exactly; attention outputs on sampled Q tiles of sampled heads
     (first, last / ragged tail, random) checked element by element."""
     w = W.get(name)
     q, k, v = W.make_qkv(w)
-    p, ws, view, o = gpu_attention(w, q, k, v)
+    p, ws, view, o = gpu_attention(w, q, k, v, PV_MODES[mode])
     quant = oracle_quant(w, q, k, v)
     bad = compare_quant(w, p, ws, view, quant)
     assert not bad, bad
@@ -141,3 +156,16 @@ def test_full_size_quant_bit_exact_and_sampled_attention(name):
     for (b, h, r0, r1), ref in zip(jobs, refs):
         m, ok = compare_out(ref, out[b, h, r0:r1])
         assert ok, ((b, h, r0, r1), m)
+
+
+def test_fp8_accumulator_precision_probe():
+    """The two-level accumulation of SageAttention2 exists because Ada/Hopper FP8
+    MMAs keep about 13 accumulator bits (SA2 note, "5. Numerical
+    Considerations").  This runs the tcgen05 kind::f8f6f4 probe: sums that need
+    at most 12 mantissa bits must come back exact whatever the accumulator
+    width; the others show how many bits it keeps (recorded, not asserted)."""
+    got = sage.sage_debug_f8_accum_probe().cpu().numpy().astype(np.float64)
+    exact = np.array(sage.F8_ACCUM_PROBE_EXACT)
+    assert got[2] == exact[2] and got[3] == 256.0 and got[4] == 32.0, got
+    bits = [int(-np.log2(abs(g - round(g)) or 2.0 ** -40)) if g != round(g) else None for g in got]
+    print("f8 accumulator probe:", got.tolist(), "exact:", [float(x) == float(y) for x, y in zip(got, exact)], bits)
