@@ -34,6 +34,7 @@ sys.path.insert(0, _ROOT)
 from quantized_attention_block_b200 import workloads as W  # noqa: E402
 
 INT8_FP8_PER_BF16 = 2.0  # nominal dense ratio 4.5 / 2.25 PFLOP/s
+FP4_PER_BF16 = 4.0  # nominal dense ratio 9 / 2.25 PFLOP/s
 
 
 def _peaks():
@@ -154,22 +155,26 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     p = sage.make_params(qd, kd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
                          smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=pv_accum)
-    wsp = sage.alloc_workspace(p)
+    wsp = sage.alloc_nvfp4_workspace(p) if w.nvfp4 else sage.alloc_workspace(p)
     o = torch.empty_like(qd)
     stream = torch.cuda.current_stream()
+    quant = sage.sage_quant_nvfp4 if w.nvfp4 else sage.sage_quant_qkv
+    attn = sage.sage_attn_fwd_nvfp4_quantized if w.nvfp4 else sage.sage_attn_fwd_quantized
+    if w.nvfp4:
+        time_other_mode = False  # one accumulation scheme on the NVFP4 path
 
     def step(ev=None):
-        view = sage.sage_quant_qkv(qd, kd, vd, p, wsp, stream)
+        view = quant(qd, kd, vd, p, wsp, stream)
         if ev is not None:
             ev[0].record(stream)
-        sage.sage_attn_fwd_quantized(view, o, p, stream)
+        attn(view, o, p, stream)
         if ev is not None:
             ev[1].record(stream)
 
     for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
-    launches_per_step = 4 + (1 if w.smooth_q else 0)
+    launches_per_step = 4 + (1 if w.smooth_q else 0) + (1 if w.nvfp4 else 0)
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
@@ -212,9 +217,13 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
             qd.copy_(qh, non_blocking=True)
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
-            sage.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
-                               smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=pv_accum, out=o, workspace=wsp,
-                               stream=stream)
+            if w.nvfp4:
+                sage.sage_attn_fwd_nvfp4(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                                         smooth_q=w.smooth_q, bq=w.bq, out=o, workspace=wsp, stream=stream)
+            else:
+                sage.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                                   smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=pv_accum, out=o,
+                                   workspace=wsp, stream=stream)
             oh.copy_(o, non_blocking=True)
 
         for _ in range(2):
@@ -274,7 +283,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sage", "reference"], default="sage")
     ap.add_argument("--workload", default="prefill")
-    ap.add_argument("--extra-workloads", default="video,gqa")
+    ap.add_argument("--extra-workloads", default="video,gqa,nvfp4")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--override", default="", help="workload fields, e.g. B=1,Hq=16,Hkv=16 (profiling cases)")
@@ -336,12 +345,16 @@ def main():
         we = W.get(name)
         me = pv_mode(we, args.pv_accum)
         r = run_sage(we, max(3, args.steps // 4), 3, ws, rank, local, False, me, time_other_mode=True)
-        extra[we.name] = {"pv_accum": ["two_level", "tmem_fp32"][me],
+        pk = peaks["bf16_tflops_sustained"] * (FP4_PER_BF16 if we.nvfp4 else INT8_FP8_PER_BF16)
+        extra[we.name] = {"pv_accum": "scaled_tmem_fp32" if we.nvfp4 else ["two_level", "tmem_fp32"][me],
+                          "path": "nvfp4" if we.nvfp4 else "int8_fp8",
                           "step_tops": we.ops() / (r["ms_step"] * 1e-3) / 1e12,
-                          "attn_kernel_tops_other_mode": we.ops() / (r["ms_attn_other_mode"] * 1e-3) / 1e12,
                           "attn_kernel_tops": we.ops() / (r["ms_attn"] * 1e-3) / 1e12,
                           "ms_step": r["ms_step"], "ms_attn": r["ms_attn"],
-                          "attn_frac_of_peak": we.ops() / (r["ms_attn"] * 1e-3) / 1e12 / peak_tops}
+                          "attn_frac_of_peak": we.ops() / (r["ms_attn"] * 1e-3) / 1e12 / pk,
+                          "peak_tops": pk}
+        if "ms_attn_other_mode" in r:
+            extra[we.name]["attn_kernel_tops_other_mode"] = we.ops() / (r["ms_attn_other_mode"] * 1e-3) / 1e12
     line = {
         "metric": metric, "value": value, "unit": "TOPS", "n_gpus": ws, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": res["ms_step"], "higher_is_better": True,

@@ -202,6 +202,72 @@ SAGE_API sage_status sage_attn_fwd_noalloc(const void *q, const void *k, const v
  */
 SAGE_API sage_status sage_debug_f8_accum_probe(float *out8, void *stream);
 
+/*
+ * ---------------------------------------------------------------- NVFP4 path
+ * SageAttention3 reading note (zhaifeiyue.github.io/papers/2505.11594),
+ * "Microscaling FP4 attention" and the two-level quantisation of P.  Same
+ * sage_params (d must be 128; bq is the smooth-Q block, 64 or 128; bk and
+ * pv_accum are not used).  E2M1 codes are packed two per byte, the even
+ * element in the low nibble; every 16 consecutive elements share one E4M3
+ * scale E4M3(amax16 / 6).  Scale blocks hold, per 128-row tile, two 512-byte
+ * blocks (64-element K chunks kk = 0, 1); in block kk the scale of row m
+ * (Q row, key, or V channel) for its 16-element group 4 kk + k is at byte
+ * 16 (m % 32) + 4 (m / 32) + k.  Padded rows hold zero codes and scales.
+ */
+typedef struct {
+    uint8_t *q4;   /* [B, Hq,  Np, d/2]        E2M1 of (Q - qbar) or Q, along d       */
+    uint8_t *k4;   /* [B, Hkv, Np, d/2]        E2M1 of gamma(K) = K - km, along d     */
+    uint8_t *v4t;  /* [B, Hkv, d, Np/2]        E2M1 of V along tokens, transposed     */
+    uint8_t *sfq;  /* [B, Hq,  Np/128, 1024]   E4M3 scales of q4 (16 channels each)   */
+    uint8_t *sfk;  /* [B, Hkv, Np/128, 1024]   E4M3 scales of k4                      */
+    uint8_t *sfv;  /* [B, Hkv, Np/128, 1024]   E4M3 scales of v4t (16 tokens each)    */
+    float   *km;   /* [B, Hkv, d]              mean(K) over tokens (zeros if !smooth_k) */
+    float   *qbar; /* [B, Hq,  Tm, d]          Q block means (NULL unless smooth_q)   */
+    float   *dS;   /* [B, Hq,  Tm, Np]         delta_S = qbar . gamma(K)^T (or NULL)  */
+    int64_t  Np;
+} sage_nvfp4_view;
+
+/* Workspace bytes the NVFP4 entry points need for `p` (0 if p is invalid or d != 128). */
+SAGE_API size_t sage_nvfp4_workspace_bytes(const sage_params *p);
+
+/*
+ * NVFP4 preprocessing: km, gamma(K) and (smooth_q) qbar / delta_S exactly as
+ * sage_quant_qkv; then per 16-element group sb = E4M3_rn_satfinite(amax / 6)
+ * (IEEE fp32 division) and codes E2M1_rn_satfinite(x / sb) (0 when sb == 0),
+ * along d for Q and K and along tokens for V.  Bit-exact with these
+ * definitions.  Fills *view with pointers into `workspace`.
+ */
+SAGE_API sage_status sage_quant_nvfp4(const void *q, const void *k, const void *v, const sage_params *p,
+                                      void *workspace, size_t workspace_bytes, sage_nvfp4_view *view,
+                                      void *stream);
+
+/*
+ * The fused NVFP4 attention kernel on a view from sage_quant_nvfp4 (same p):
+ * S = (Q^ sq)(K^ sk)^T (+ dS), scaled by sm_scale (tcgen05 kind::mxf4nvf4);
+ * online softmax in FP32; per row and key tile s_P1 = rowmax(P~) / 2688,
+ * P2 = P~ / s_P1, s_P2 = E4M3(amax16(P2) / 6), P^ = E2M1(P2 / s_P2); the
+ * block-scaled P^ V^ product is accumulated in FP32 with the s_P1 and
+ * exp(m_old - m) factors; o = O / l in p->dtype, [B, Hq, N, d].
+ */
+SAGE_API sage_status sage_attn_fwd_nvfp4_quantized(const sage_nvfp4_view *view, void *o, const sage_params *p,
+                                                   void *stream);
+
+/* sage_quant_nvfp4 followed by sage_attn_fwd_nvfp4_quantized. */
+SAGE_API sage_status sage_attn_fwd_nvfp4(const void *q, const void *k, const void *v, void *o,
+                                         const sage_params *p, void *workspace, size_t workspace_bytes,
+                                         void *stream);
+
+/*
+ * Probe of the block-scaled FP4 tensor-core path: the FP32 tile
+ * (Q^ sq)(K^ sk)^T (no delta_S, no sm_scale) for rows [128 qtile, +128) of
+ * head (b, h) and keys [128 ktile, +128), through the same TMA staging,
+ * scale-block copies and MMA as the attention kernel; row-major to
+ * out_128x128 (device, 128*128 floats).
+ */
+SAGE_API sage_status sage_debug_qk_nvfp4(const sage_nvfp4_view *view, const sage_params *p, int32_t b,
+                                         int32_t h, int32_t qtile, int32_t ktile, float *out_128x128,
+                                         void *stream);
+
 /* Human-readable name of a status code (static storage). */
 SAGE_API const char *sage_status_string(sage_status s);
 

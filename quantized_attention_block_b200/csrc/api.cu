@@ -190,6 +190,94 @@ AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d
 
 sage_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
 
+// ---------------------------------------------------------------- NVFP4 layout
+struct LayoutF4 {
+  size_t q4, k4, v4t, sfq, sfk, sfv, km, ksum, qbar, dS, total;
+};
+
+LayoutF4 make_layout_f4(const sage_params* p, const Dims& d) {
+  LayoutF4 L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  const size_t tiles = (size_t)(d.Np / kTile);
+  L.q4 = take((size_t)(d.B * d.Hq * d.Np * d.D / 2));
+  L.k4 = take((size_t)(d.B * d.Hkv * d.Np * d.D / 2));
+  L.v4t = take((size_t)(d.B * d.Hkv * d.D * d.Np / 2));
+  L.sfq = take((size_t)(d.B * d.Hq) * tiles * 1024);
+  L.sfk = take((size_t)(d.B * d.Hkv) * tiles * 1024);
+  L.sfv = take((size_t)(d.B * d.Hkv) * tiles * 1024);
+  L.km = take(4 * (size_t)(d.B * d.Hkv * d.D));
+  L.ksum = take(8 * (size_t)(d.B * d.Hkv * d.D));
+  if (p->smooth_q) {
+    L.qbar = take(4 * (size_t)(d.B * d.Hq * d.Tm * d.D));
+    L.dS = take(4 * (size_t)(d.B * d.Hq * d.Tm * d.Np));
+  }
+  L.total = off;
+  return L;
+}
+
+sage_status check_params_f4(const sage_params* p, Dims* d) {
+  const sage_status s = check_params(p, d);
+  if (s != SAGE_OK) return s;
+  return d->D == 128 ? SAGE_OK : SAGE_ERR_UNSUPPORTED_HEADDIM;
+}
+
+void fill_view_f4(const sage_params* p, const Dims& d, void* ws, sage_nvfp4_view* v) {
+  const LayoutF4 L = make_layout_f4(p, d);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  v->q4 = base + L.q4;
+  v->k4 = base + L.k4;
+  v->v4t = base + L.v4t;
+  v->sfq = base + L.sfq;
+  v->sfk = base + L.sfk;
+  v->sfv = base + L.sfv;
+  v->km = reinterpret_cast<float*>(base + L.km);
+  v->qbar = p->smooth_q ? reinterpret_cast<float*>(base + L.qbar) : nullptr;
+  v->dS = p->smooth_q ? reinterpret_cast<float*>(base + L.dS) : nullptr;
+  v->Np = d.Np;
+}
+
+// Q / K: rows of 64 bytes (128 E2M1 codes); V^T: rows of Np/2 bytes.  Boxes
+// of 64 bytes x 128 rows, 64-byte swizzle (the MMA's K-major SW64 layout).
+sage_status make_maps_f4(const sage_nvfp4_view* v, const Dims& d, CUtensorMap* mQ, CUtensorMap* mK,
+                         CUtensorMap* mV) {
+  const CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!map_2d_u8(mQ, v->q4, 64, (uint64_t)(d.B * d.Hq * d.Np), 64, kTile, swz)) return SAGE_ERR_CUDA;
+  if (!map_2d_u8(mK, v->k4, 64, (uint64_t)(d.B * d.Hkv * d.Np), 64, kTile, swz)) return SAGE_ERR_CUDA;
+  if (mV && !map_2d_u8(mV, v->v4t, (uint64_t)(d.Np / 2), (uint64_t)(d.B * d.Hkv * d.D), 64, kTile, swz))
+    return SAGE_ERR_CUDA;
+  return SAGE_OK;
+}
+
+AttnArgs attn_args_f4(const sage_nvfp4_view* v, const sage_params* p, const Dims& d) {
+  AttnArgs a{};
+  a.B = (int)d.B;
+  a.Hq = (int)d.Hq;
+  a.Hkv = (int)d.Hkv;
+  a.N = (int)d.N;
+  a.D = (int)d.D;
+  a.Np = d.Np;
+  a.Tm = (int)d.Tm;
+  a.Tn = (int)d.Tn;
+  a.bq = p->bq;
+  a.bk = p->bk;
+  a.causal = p->causal;
+  a.n_qtiles = (int)(d.Np / kTile);
+  const float sm = p->sm_scale > 0.0f ? p->sm_scale : 1.0f / std::sqrt((float)d.D);
+  a.scale_log2 = (float)((double)sm * 1.4426950408889634);
+  a.dS = p->smooth_q ? v->dS : nullptr;
+  a.out_fp16 = p->dtype == SAGE_FP16;
+  a.sfq = v->sfq;
+  a.sfk = v->sfk;
+  a.sfv = v->sfv;
+  return a;
+}
+
+
 
 }  // namespace
 
@@ -293,6 +381,101 @@ sage_status sage_debug_qk_int32(const sage_quant_view* view, const sage_params* 
   a.probe_ktile = ktile;
   a.probe_out = out;
   return from_cuda(launch_qk_probe(a, mQ, mK, static_cast<cudaStream_t>(stream)));
+}
+
+size_t sage_nvfp4_workspace_bytes(const sage_params* p) {
+  Dims d;
+  if (check_params_f4(p, &d) != SAGE_OK) return 0;
+  return make_layout_f4(p, d).total;
+}
+
+sage_status sage_quant_nvfp4(const void* q, const void* k, const void* v, const sage_params* p, void* workspace,
+                             size_t workspace_bytes, sage_nvfp4_view* view, void* stream) {
+  Dims d;
+  sage_status s = check_params_f4(p, &d);
+  if (s != SAGE_OK) return s;
+  if (!q || !k || !v || !workspace || !view) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SAGE_ERR_MISALIGNED;
+  const LayoutF4 L = make_layout_f4(p, d);
+  if (workspace_bytes < L.total) return SAGE_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_arch()) != SAGE_OK) return s;
+  fill_view_f4(p, d, workspace, view);
+  QuantArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.B = (int)d.B;
+  a.Hq = (int)d.Hq;
+  a.Hkv = (int)d.Hkv;
+  a.N = (int)d.N;
+  a.D = (int)d.D;
+  a.Np = d.Np;
+  a.Tm = (int)d.Tm;
+  a.Tn = (int)d.Tn;
+  a.bq = p->bq;
+  a.bk = p->bk;
+  a.smooth_k = p->smooth_k;
+  a.smooth_q = p->smooth_q;
+  a.km = view->km;
+  a.qbar = view->qbar;
+  a.dS = view->dS;
+  a.ksum = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + L.ksum);
+  a.q4 = view->q4;
+  a.k4 = view->k4;
+  a.v4t = view->v4t;
+  a.sfq = view->sfq;
+  a.sfk = view->sfk;
+  a.sfv = view->sfv;
+  return from_cuda(launch_quant_nvfp4(a, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status sage_attn_fwd_nvfp4_quantized(const sage_nvfp4_view* view, void* o, const sage_params* p,
+                                          void* stream) {
+  Dims d;
+  sage_status s = check_params_f4(p, &d);
+  if (s != SAGE_OK) return s;
+  if (!view || !o || !view->q4 || !view->k4 || !view->v4t || !view->sfq || !view->sfk || !view->sfv)
+    return SAGE_ERR_INVALID_ARG;
+  if (p->smooth_q && !view->dS) return SAGE_ERR_INVALID_ARG;
+  if (view->Np != d.Np) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(view->q4) || !aligned16(view->k4) || !aligned16(view->v4t) ||
+      !aligned16(view->sfq) || !aligned16(view->sfk) || !aligned16(view->sfv))
+    return SAGE_ERR_MISALIGNED;
+  if ((s = check_arch()) != SAGE_OK) return s;
+  CUtensorMap mQ, mK, mV;
+  if ((s = make_maps_f4(view, d, &mQ, &mK, &mV)) != SAGE_OK) return s;
+  AttnArgs a = attn_args_f4(view, p, d);
+  a.o = o;
+  return from_cuda(launch_attn_nvfp4(a, mQ, mK, mV, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status sage_attn_fwd_nvfp4(const void* q, const void* k, const void* v, void* o, const sage_params* p,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  sage_nvfp4_view view;
+  sage_status s = sage_quant_nvfp4(q, k, v, p, workspace, workspace_bytes, &view, stream);
+  if (s != SAGE_OK) return s;
+  return sage_attn_fwd_nvfp4_quantized(&view, o, p, stream);
+}
+
+sage_status sage_debug_qk_nvfp4(const sage_nvfp4_view* view, const sage_params* p, int32_t b, int32_t h,
+                                int32_t qtile, int32_t ktile, float* out, void* stream) {
+  Dims d;
+  sage_status s = check_params_f4(p, &d);
+  if (s != SAGE_OK) return s;
+  if (!view || !out || !view->q4 || !view->k4 || !view->sfq || !view->sfk) return SAGE_ERR_INVALID_ARG;
+  if (b < 0 || b >= d.B || h < 0 || h >= d.Hq || qtile < 0 || ktile < 0 || qtile >= d.Np / kTile ||
+      ktile >= d.Np / kTile)
+    return SAGE_ERR_INVALID_ARG;
+  if ((s = check_arch()) != SAGE_OK) return s;
+  CUtensorMap mQ, mK;
+  if ((s = make_maps_f4(view, d, &mQ, &mK, nullptr)) != SAGE_OK) return s;
+  AttnArgs a = attn_args_f4(view, p, d);
+  a.probe_b = b;
+  a.probe_h = h;
+  a.probe_qtile = qtile;
+  a.probe_ktile = ktile;
+  return from_cuda(launch_qk_probe_nvfp4(a, mQ, mK, out, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status sage_last_device_error(void* stream) {

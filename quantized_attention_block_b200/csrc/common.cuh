@@ -28,7 +28,16 @@ struct QuantArgs {
   float* qbar;
   float* dS;
   double* ksum;     // [B,Hkv,D] fp64 column sums of K
-  unsigned* vamax;  // [B,Hkv,D] bit pattern of max |V| (non-negative floats order as uints)
+  unsigned* vamax;  // [B,Hkv,D] bit pattern of max |V| (non-negative floats order as uints);
+                    // nullptr: the statistics pass skips V (NVFP4 path)
+  // NVFP4 path (E2M1 codes two per byte, low nibble first; 1 KB scale blocks
+  // per 128-row tile in the tcgen05 scale-factor order)
+  uint8_t* q4;   // [B,Hq,Np,D/2]
+  uint8_t* k4;   // [B,Hkv,Np,D/2]
+  uint8_t* v4t;  // [B,Hkv,D,Np/2]
+  uint8_t* sfq;  // [B,Hq,Np/128,1024]
+  uint8_t* sfk;  // [B,Hkv,Np/128,1024]
+  uint8_t* sfv;  // [B,Hkv,Np/128,1024]
 };
 
 struct AttnArgs {
@@ -46,6 +55,10 @@ struct AttnArgs {
   int out_fp16;
   int two_level;  // 1: fresh O_t per key tile + FP32 add on CUDA cores; 0: TMEM FP32 accumulator
   int pingpong;   // 1: the two softmax warpgroups take turns; 0: they run concurrently
+  // NVFP4 scale blocks (1 KB per 128-row tile)
+  const uint8_t* sfq;
+  const uint8_t* sfk;
+  const uint8_t* sfv;
   // probe mode (sage_debug_qk_int32)
   int probe_b, probe_h, probe_qtile, probe_ktile;
   int32_t* probe_out;
@@ -58,5 +71,10 @@ cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CU
 cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(cudaStream_t st);
 cudaError_t launch_f8_accum_probe(float* out, cudaStream_t st);
+cudaError_t launch_quant_nvfp4(const QuantArgs& a, int is_fp16, cudaStream_t st);
+cudaError_t launch_attn_nvfp4(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                              const CUtensorMap& tmV, cudaStream_t st);
+cudaError_t launch_qk_probe_nvfp4(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                  float* out, cudaStream_t st);
 
 }  // namespace sage

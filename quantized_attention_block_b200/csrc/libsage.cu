@@ -3,5 +3,7 @@
 // device code).
 #include "quant.cu"
 #include "attn_i8f8.cu"
+#include "quant_nvfp4.cu"
+#include "attn_nvfp4.cu"
 #include "api.cu"
 #include "noalloc.cu"

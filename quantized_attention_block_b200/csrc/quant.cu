@@ -92,7 +92,8 @@ __device__ __forceinline__ float block_max_nonneg(float v, float* red) {
 }
 
 // ---------------------------------------------------------------------------
-// Pass 1: per (b, kv-head, channel) fp64 sum of K (smooth K) and max |V|.
+// Pass 1: per (b, kv-head, channel) fp64 sum of K (smooth K) and max |V|
+// (skipped when a.vamax is null).
 // grid (ceil(N / kStatRows), B*Hkv)
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
@@ -114,9 +115,11 @@ __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
     load8<T>(K + r * D + ch * 8, x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) ks[e] += (double)x[e];
-    load8<T>(V + r * D + ch * 8, x);
+    if (a.vamax) {
+      load8<T>(V + r * D + ch * 8, x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) va[e] = fmaxf(va[e], fabsf(x[e]));
+      for (int e = 0; e < 8; ++e) va[e] = fmaxf(va[e], fabsf(x[e]));
+    }
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) { s_sum[threadIdx.x][e] = ks[e]; s_amax[threadIdx.x][e] = va[e]; }
@@ -130,7 +133,7 @@ __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
       m = fmaxf(m, s_amax[g * CH + c / 8][c % 8]);
     }
     if (a.smooth_k) atomicAdd(&a.ksum[(int64_t)bg * D + c], s);
-    atomicMax(&a.vamax[(int64_t)bg * D + c], __float_as_uint(m));
+    if (a.vamax) atomicMax(&a.vamax[(int64_t)bg * D + c], __float_as_uint(m));
   }
 }
 

@@ -1,0 +1,261 @@
+// quant_nvfp4.cu -- NVFP4 preprocessing on sm_100a (HBM-bound kernels).
+//
+// SageAttention3 as summarised in its reading note
+// (zhaifeiyue.github.io/papers/2505.11594), "Microscaling FP4 attention": Q and
+// K are smoothed (K by its token mean, Q by its per-block mean with the delta_S
+// compensation of SageAttention2), then every group of 16 consecutive elements
+// along the head dimension gets one E4M3 scale, sb = E4M3(amax16 / 6), and E2M1
+// codes E2M1(x / sb).  V is grouped the same way along tokens (the reduction
+// axis of P V).  Every division is an IEEE fp32 division (__fdiv_rn); E2M1 and
+// E4M3 use round-to-nearest-even with saturation (cvt.rn.satfinite), so codes
+// and scales are bit-exact with the plain definitions.
+//
+// Output layouts (what the attention kernel's TMA / bulk copies read):
+//   q4 [B,Hq,Np,64], k4 [B,Hkv,Np,64]: E2M1 codes of a row, two per byte, the
+//     even element in the low nibble.
+//   v4t [B,Hkv,128,Np/2]: V transposed, codes along tokens, same packing.
+//   sfq / sfk / sfv [.., Np/128, 1024]: per 128-row tile, two 512-byte blocks
+//     (K chunks of 64 elements); in block kk the scale of row m (Q row, key, or
+//     V channel) for its 16-element group kk*4 + k sits at byte
+//     16 (m % 32) + 4 (m / 32) + k -- the order tcgen05.cp broadcasts into TMEM.
+// Only head_dim 128 is supported on this path.
+
+namespace sage {
+
+namespace {
+
+constexpr int kF4D = 128;
+
+__device__ __forceinline__ int sf_byte(int m, int grp) {
+  return (grp >> 2) * 512 + 16 * (m & 31) + 4 * (m >> 5) + (grp & 3);
+}
+
+// E2M1 codes of x / sd for 8 values (0 when sd == 0), packed low nibble first.
+__device__ __forceinline__ uint32_t encode8_e2m1(const float (&x)[8], float sd) {
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] = sd == 0.0f ? 0.0f : __fdiv_rn(x[e], sd);
+  return cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+}
+
+// Encodes row chunk x (8 channels) of a 16-group shared with the partner lane
+// (lane ^ 1): returns the 4 code bytes, writes the group's scale code to *sc.
+__device__ __forceinline__ uint32_t encode_pair(const float (&x)[8], uint32_t* sc) {
+  float am = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x[e]));
+  am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+  const uint32_t c = cvt_e4m3(__fdiv_rn(am, 6.0f));
+  *sc = c;
+  return encode8_e2m1(x, e4m3_value(c));
+}
+
+// ---------------------------------------------------------------------------
+// K: gamma(K) = K - km, NVFP4 along d.  grid (Np/128, B*Hkv), 256 threads.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_quant_nvfp4_kernel(QuantArgs a) {
+  constexpr int D = kF4D, CH = D / 8, RG = kThreads / CH, NP = kTile / RG;
+  __shared__ float s_km[D];
+  __shared__ __align__(16) uint8_t s_sf[1024];
+  const int bg = blockIdx.y, tile = blockIdx.x;
+  const int64_t r0 = (int64_t)tile * kTile;
+  const int valid = rows_valid(a.N, r0, kTile);
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    const float km = a.smooth_k ? __double2float_rn(__ddiv_rn(a.ksum[(int64_t)bg * D + c], (double)a.N)) : 0.0f;
+    s_km[c] = km;
+    if (tile == 0) a.km[(int64_t)bg * D + c] = km;
+  }
+  __syncthreads();
+  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
+  uint8_t* k4 = a.k4 + ((int64_t)bg * a.Np + r0) * (D / 2);
+#pragma unroll 2
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    float x[8];
+    if (r < valid) {
+      load8<T>(K + (r0 + r) * D + ch * 8, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], s_km[ch * 8 + e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+    }
+    uint32_t sc;
+    const uint32_t codes = encode_pair(x, &sc);
+    *reinterpret_cast<uint32_t*>(k4 + r * (D / 2) + ch * 4) = codes;
+    if ((ch & 1) == 0) s_sf[sf_byte(r, ch >> 1)] = (uint8_t)sc;
+  }
+  __syncthreads();
+  reinterpret_cast<uint32_t*>(a.sfk + ((int64_t)bg * (a.Np / kTile) + tile) * 1024)[threadIdx.x] =
+      reinterpret_cast<const uint32_t*>(s_sf)[threadIdx.x];
+}
+
+// ---------------------------------------------------------------------------
+// Q: optional per-BQ-block mean (smooth Q), NVFP4 along d.  One 128-row tile
+// per CTA (128 / BQ mean blocks).  grid (Np/128, B*Hq), 256 threads.
+template <typename T, int BQ>
+__global__ void __launch_bounds__(kThreads) q_quant_nvfp4_kernel(QuantArgs a) {
+  constexpr int D = kF4D, CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BQ, PPB = BQ / RG;
+  __shared__ double s_sum[kThreads][8];
+  __shared__ float s_mean[NB][D];
+  __shared__ __align__(16) uint8_t s_sf[1024];
+  const int bh = blockIdx.y, tile = blockIdx.x;
+  const int64_t r0 = (int64_t)tile * kTile;
+  const int valid = rows_valid(a.N, r0, kTile);
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  const T* Q = reinterpret_cast<const T*>(a.q) + (int64_t)bh * a.N * D;
+  float x[NP][8];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    if (r < valid) {
+      load8<T>(Q + (r0 + r) * D + ch * 8, x[p]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[p][e] = 0.0f;
+    }
+  }
+  if (a.smooth_q) {
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
+      double cs[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+      for (int p = nb * PPB; p < (nb + 1) * PPB; ++p)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cs[e] += (double)x[p][e];  // invalid rows hold 0
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
+      __syncthreads();
+      if (threadIdx.x < D) {
+        const int c = threadIdx.x;
+        double s = 0.0;
+        for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
+        const float mu = vb > 0 ? __double2float_rn(__ddiv_rn(s, (double)vb)) : 0.0f;
+        s_mean[nb][c] = mu;
+        const int blk = tile * NB + nb;
+        if (vb > 0) a.qbar[((int64_t)bh * a.Tm + blk) * D + c] = mu;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int p = 0; p < NP; ++p)
+      if (rg + p * RG < valid)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[p][e] = __fsub_rn(x[p][e], s_mean[p / PPB][ch * 8 + e]);
+  }
+  uint8_t* q4 = a.q4 + ((int64_t)bh * a.Np + r0) * (D / 2);
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    uint32_t sc;
+    const uint32_t codes = encode_pair(x[p], &sc);
+    *reinterpret_cast<uint32_t*>(q4 + r * (D / 2) + ch * 4) = codes;
+    if ((ch & 1) == 0) s_sf[sf_byte(r, ch >> 1)] = (uint8_t)sc;
+  }
+  __syncthreads();
+  reinterpret_cast<uint32_t*>(a.sfq + ((int64_t)bh * (a.Np / kTile) + tile) * 1024)[threadIdx.x] =
+      reinterpret_cast<const uint32_t*>(s_sf)[threadIdx.x];
+}
+
+// ---------------------------------------------------------------------------
+// V: NVFP4 along tokens (16-token groups per channel), transposed to
+// [D][Np/2].  The tile is staged in shared memory; each thread encodes one
+// (channel, 16-token group) at a time, consecutive threads taking consecutive
+// channels; codes go through shared memory so the global stores are 16-byte
+// rows.  grid (Np/128, B*Hkv), 256 threads.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) v_quant_nvfp4_kernel(QuantArgs a) {
+  constexpr int D = kF4D, CH = D / 8, RG = kThreads / CH, NP = kTile / RG, kPitch = D + 8;
+  __shared__ __align__(16) T sV[kTile * kPitch];
+  __shared__ __align__(16) uint8_t sVt[D * (kTile / 2)];
+  __shared__ __align__(16) uint8_t s_sf[1024];
+  const int bg = blockIdx.y, tile = blockIdx.x;
+  const int64_t r0 = (int64_t)tile * kTile;
+  const int valid = rows_valid(a.N, r0, kTile);
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)bg * a.N * D;
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int r = rg + p * RG;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (r < valid) u = __ldg(reinterpret_cast<const uint4*>(V + (r0 + r) * D + ch * 8));
+    *reinterpret_cast<uint4*>(sV + r * kPitch + ch * 8) = u;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < (D * 8) / kThreads; ++it) {
+    const int item = threadIdx.x + it * kThreads;
+    const int c = item % D, grp = item / D;
+    float x[16];
+    float am = 0.0f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      x[u] = to_float(sV[(grp * 16 + u) * kPitch + c]);
+      am = fmaxf(am, fabsf(x[u]));
+    }
+    const uint32_t sc = cvt_e4m3(__fdiv_rn(am, 6.0f));
+    const float sd = e4m3_value(sc);
+    float lo[8], hi[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      lo[u] = x[u];
+      hi[u] = x[8 + u];
+    }
+    const uint2 codes = make_uint2(encode8_e2m1(lo, sd), encode8_e2m1(hi, sd));
+    *reinterpret_cast<uint2*>(sVt + c * (kTile / 2) + grp * 8) = codes;
+    s_sf[sf_byte(c, grp)] = (uint8_t)sc;
+  }
+  __syncthreads();
+  uint8_t* v4t = a.v4t + (int64_t)bg * D * (a.Np / 2) + r0 / 2;
+#pragma unroll
+  for (int it = 0; it < (D * kTile / 2 / 16) / kThreads; ++it) {
+    const int idx = threadIdx.x + it * kThreads;  // 16-byte chunk
+    const int c = idx / 4, q = idx % 4;
+    *reinterpret_cast<uint4*>(v4t + (int64_t)c * (a.Np / 2) + q * 16) =
+        *reinterpret_cast<const uint4*>(sVt + c * (kTile / 2) + q * 16);
+  }
+  reinterpret_cast<uint32_t*>(a.sfv + ((int64_t)bg * (a.Np / kTile) + tile) * 1024)[threadIdx.x] =
+      reinterpret_cast<const uint32_t*>(s_sf)[threadIdx.x];
+}
+
+template <typename T>
+cudaError_t launch_quant_nvfp4_t(const QuantArgs& a, cudaStream_t st) {
+  cudaError_t e;
+  const int BHkv = a.B * a.Hkv, BHq = a.B * a.Hq;
+  const int tiles = (int)(a.Np / kTile);
+  QuantArgs s = a;
+  s.vamax = nullptr;  // no per-channel V statistics on this path
+  if (a.smooth_k) {
+    e = cudaMemsetAsync(a.ksum, 0, sizeof(double) * (size_t)BHkv * kF4D, st);
+    if (e != cudaSuccess) return e;
+  }
+  kv_stats_kernel<T, kF4D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(s);
+  k_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, 0, st>>>(s);
+  v_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, 0, st>>>(s);
+  if (a.bq == 64)
+    q_quant_nvfp4_kernel<T, 64><<<dim3(tiles, BHq), kThreads, 0, st>>>(s);
+  else
+    q_quant_nvfp4_kernel<T, 128><<<dim3(tiles, BHq), kThreads, 0, st>>>(s);
+  if (a.smooth_q) {
+    const size_t smem = sizeof(float) * kF4D * kTile;
+    e = cudaFuncSetAttribute(delta_s_kernel<T, kF4D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    delta_s_kernel<T, kF4D><<<dim3(tiles, BHq), kThreads, smem, st>>>(s);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quant_nvfp4(const QuantArgs& a, int is_fp16, cudaStream_t st) {
+  if (a.D != kF4D) return cudaErrorInvalidValue;
+  return is_fp16 ? launch_quant_nvfp4_t<__half>(a, st) : launch_quant_nvfp4_t<__nv_bfloat16>(a, st);
+}
+
+}  // namespace sage

@@ -174,6 +174,30 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint
       : "memory");
 }
 
+// D[tmem] (+)= (A * sfA)[smem] * (B * sfB)[smem]^T: packed E2M1 (NVFP4) inputs
+// with one UE4M3 scale per 16 elements along K, f32 accumulator.  One
+// instruction covers K = 64; the scale factors of A and B are read from TMEM
+// at columns sfa / sfb (4 columns each for 128 rows: see tmem_cp_sf).
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared -> TMEM copy of one 512-byte scale-factor block (32 rows x 16 bytes,
+// row-contiguous), broadcast to the four 32-lane sub-partitions: TMEM lane
+// 32 w + r, columns [col, col + 4) receive row r.  For a 128-row operand the
+// block holds row m = 32 q + r's four scales (K = 64) at byte 16 r + 4 q + k,
+// which is the order the block-scaled MMA reads them in.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive on `bar` once all previously issued tcgen05 async ops of this thread finish.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -269,6 +293,12 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t sbo_byte
   return d;
 }
 
+// Instruction descriptor for kind::mxf4nvf4 with block16 UE4M3 scales:
+// A and B E2M1 (format 1), K-major, scale format 0 (UE4M3), scale ids 0, K = 64.
+__host__ __device__ constexpr uint32_t make_idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Instruction descriptor for kind::f16 / tf32 / f8f6f4 / i8 (dense, K-major A and B).
 //   c_fmt: 0 F16, 1 F32, 2 S32;  a/b_fmt: kind-specific (i8: 1 = signed; f8f6f4: 0 = E4M3)
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t c_fmt, uint32_t a_fmt, uint32_t b_fmt, int M, int N) {
@@ -305,6 +335,41 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Eight floats -> eight E2M1 codes (round-to-nearest-even, saturate to +-6),
+// element e in bits [4e, 4e + 4).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float f0, float f1, float f2, float f3, float f4, float f5, float f6,
+                                               float f7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(f0), "f"(f1), "f"(f2), "f"(f3), "f"(f4), "f"(f5), "f"(f6), "f"(f7));
+  return r;
+}
+
+// One float -> E4M3 code (round-to-nearest-even, saturate to +-448).
+__device__ __forceinline__ uint32_t cvt_e4m3(float x) { return cvt_e4m3x2(x, 0.0f) & 0xFFu; }
+
+// Value of a non-negative E4M3 code (exact): exponent field 0 is subnormal
+// (m * 2^-9), otherwise (8 + m) * 2^(e - 10).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
+}
+
+// 1D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 }  // namespace sage

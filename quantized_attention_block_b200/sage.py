@@ -25,7 +25,9 @@ STATUS_NAMES = {
 }
 EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd",
             "sage_debug_qk_int32", "sage_last_device_error", "sage_debug_bounded_wait",
-            "sage_status_string", "sage_attn_fwd_noalloc", "sage_debug_f8_accum_probe")
+            "sage_status_string", "sage_attn_fwd_noalloc", "sage_debug_f8_accum_probe",
+            "sage_nvfp4_workspace_bytes", "sage_quant_nvfp4", "sage_attn_fwd_nvfp4_quantized",
+            "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4")
 
 
 class SageError(RuntimeError):
@@ -52,6 +54,13 @@ class SageQuantView(ctypes.Structure):
                 ("Np", ctypes.c_int64)]
 
 
+class SageNvfp4View(ctypes.Structure):
+    _fields_ = [("q4", ctypes.c_void_p), ("k4", ctypes.c_void_p), ("v4t", ctypes.c_void_p),
+                ("sfq", ctypes.c_void_p), ("sfk", ctypes.c_void_p), ("sfv", ctypes.c_void_p),
+                ("km", ctypes.c_void_p), ("qbar", ctypes.c_void_p), ("dS", ctypes.c_void_p),
+                ("Np", ctypes.c_int64)]
+
+
 _lib = None
 
 
@@ -74,8 +83,15 @@ def lib() -> ctypes.CDLL:
         L.sage_status_string.argtypes, L.sage_status_string.restype = [ctypes.c_int], ctypes.c_char_p
         L.sage_attn_fwd_noalloc.argtypes, L.sage_attn_fwd_noalloc.restype = [vp, vp, vp, vp, P, vp], ctypes.c_int
         L.sage_debug_f8_accum_probe.argtypes, L.sage_debug_f8_accum_probe.restype = [vp, vp], ctypes.c_int
+        F = ctypes.POINTER(SageNvfp4View)
+        L.sage_nvfp4_workspace_bytes.argtypes, L.sage_nvfp4_workspace_bytes.restype = [P], ctypes.c_size_t
+        L.sage_quant_nvfp4.argtypes = [vp, vp, vp, P, vp, ctypes.c_size_t, F, vp]
+        L.sage_attn_fwd_nvfp4_quantized.argtypes = [F, vp, P, vp]
+        L.sage_attn_fwd_nvfp4.argtypes = [vp, vp, vp, vp, P, vp, ctypes.c_size_t, vp]
+        L.sage_debug_qk_nvfp4.argtypes = [F, P, i32, i32, i32, i32, vp, vp]
         for n in ("sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd", "sage_debug_qk_int32",
-                  "sage_last_device_error", "sage_debug_bounded_wait"):
+                  "sage_last_device_error", "sage_debug_bounded_wait", "sage_quant_nvfp4",
+                  "sage_attn_fwd_nvfp4_quantized", "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -190,6 +206,81 @@ def view_tensors(view: SageQuantView, p: SageParams, workspace: torch.Tensor) ->
         "s_q": sl(view.s_q, 4 * B * Hq * Tm, torch.float32, (B, Hq, Tm)),
         "s_k": sl(view.s_k, 4 * B * Hkv * Tn, torch.float32, (B, Hkv, Tn)),
         "s_v": sl(view.s_v, 4 * B * Hkv * d, torch.float32, (B, Hkv, d)),
+        "km": sl(view.km, 4 * B * Hkv * d, torch.float32, (B, Hkv, d)),
+    }
+    if view.qbar:
+        out["qbar"] = sl(view.qbar, 4 * B * Hq * Tm * d, torch.float32, (B, Hq, Tm, d))
+        out["dS"] = sl(view.dS, 4 * B * Hq * Tm * Np, torch.float32, (B, Hq, Tm, Np))
+    return out
+
+
+# ---------------------------------------------------------------- NVFP4 path
+def nvfp4_workspace_bytes(p: SageParams) -> int:
+    return int(lib().sage_nvfp4_workspace_bytes(ctypes.byref(p)))
+
+
+def alloc_nvfp4_workspace(p: SageParams, device=None) -> torch.Tensor:
+    n = nvfp4_workspace_bytes(p)
+    if n == 0:
+        raise SageError(1, "sage_nvfp4_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sage_quant_nvfp4(q, k, v, p: SageParams, workspace: torch.Tensor, stream=None) -> SageNvfp4View:
+    view = SageNvfp4View()
+    _check(lib().sage_quant_nvfp4(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(p), _ptr(workspace),
+                                  workspace.numel(), ctypes.byref(view), _stream(stream)), "sage_quant_nvfp4")
+    return view
+
+
+def sage_attn_fwd_nvfp4_quantized(view: SageNvfp4View, o: torch.Tensor, p: SageParams,
+                                  stream=None) -> torch.Tensor:
+    _check(lib().sage_attn_fwd_nvfp4_quantized(ctypes.byref(view), _ptr(o), ctypes.byref(p), _stream(stream)),
+           "sage_attn_fwd_nvfp4_quantized")
+    return o
+
+
+def sage_attn_fwd_nvfp4(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = None,
+                        smooth_k: bool = True, smooth_q: bool = True, bq: int = 128,
+                        out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """SageAttention3-style NVFP4 forward: [B,Hq,N,128] x [B,Hkv,N,128] -> [B,Hq,N,128]."""
+    p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq)
+    if workspace is None:
+        workspace = alloc_nvfp4_workspace(p, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sage_attn_fwd_nvfp4(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(p), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)), "sage_attn_fwd_nvfp4")
+    return out
+
+
+def sage_debug_qk_nvfp4(view: SageNvfp4View, p: SageParams, b: int, h: int, qtile: int, ktile: int,
+                        stream=None) -> torch.Tensor:
+    out = torch.empty((128, 128), dtype=torch.float32, device="cuda")
+    _check(lib().sage_debug_qk_nvfp4(ctypes.byref(view), ctypes.byref(p), b, h, qtile, ktile, _ptr(out),
+                                     _stream(stream)), "sage_debug_qk_nvfp4")
+    return out
+
+
+def nvfp4_view_tensors(view: SageNvfp4View, p: SageParams, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:
+    """torch views (raw device layouts) of the NVFP4 tensors inside the workspace."""
+    B, Hq, Hkv, N, d = p.B, p.Hq, p.Hkv, p.N, p.d
+    Np = int(view.Np)
+    T, Tm = Np // 128, -(-N // p.bq)
+    base = workspace.data_ptr()
+
+    def sl(ptr, nbytes, dtype, shape):
+        off = ptr - base
+        return workspace[off:off + nbytes].view(dtype).view(*shape)
+
+    out = {
+        "q4": sl(view.q4, B * Hq * Np * d // 2, torch.uint8, (B, Hq, Np, d // 2)),
+        "k4": sl(view.k4, B * Hkv * Np * d // 2, torch.uint8, (B, Hkv, Np, d // 2)),
+        "v4t": sl(view.v4t, B * Hkv * d * Np // 2, torch.uint8, (B, Hkv, d, Np // 2)),
+        "sfq": sl(view.sfq, B * Hq * T * 1024, torch.uint8, (B, Hq, T, 1024)),
+        "sfk": sl(view.sfk, B * Hkv * T * 1024, torch.uint8, (B, Hkv, T, 1024)),
+        "sfv": sl(view.sfv, B * Hkv * T * 1024, torch.uint8, (B, Hkv, T, 1024)),
         "km": sl(view.km, 4 * B * Hkv * d, torch.float32, (B, Hkv, d)),
     }
     if view.qbar:

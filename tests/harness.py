@@ -88,3 +88,102 @@ def oracle_rows(w: W.Workload, quant, b, h, r0, r1):
 def compare_out(ref: np.ndarray, out: np.ndarray):
     m = oracle.metrics(ref, out)
     return m, (m["max_abs"] <= MAX_ABS and m["cos"] >= MIN_COS and np.isfinite(out).all())
+
+
+# ---------------------------------------------------------------- NVFP4 path
+def sf_index(rows: int) -> np.ndarray:
+    """Byte offsets, inside one tile's 1 KB scale block, of scale (m, grp) for
+    m < 128, grp < 8: two 512-byte blocks (grp // 4), byte 16 (m % 32) +
+    4 (m // 32) + grp % 4 -- the device layout written by sage_quant_nvfp4."""
+    m = np.arange(rows)[:, None]
+    g = np.arange(8)[None, :]
+    return (g // 4) * 512 + 16 * (m % 32) + 4 * (m // 32) + g % 4
+
+
+def unpack_nibbles(raw: np.ndarray) -> np.ndarray:
+    """[..., n/2] bytes -> [..., n] E2M1 codes (even element in the low nibble)."""
+    out = np.empty(raw.shape[:-1] + (raw.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = raw & 15
+    out[..., 1::2] = raw >> 4
+    return out
+
+
+def unpack_sf(raw: np.ndarray) -> np.ndarray:
+    """[..., T, 1024] scale blocks -> [..., T*128, 8] scales per row and 16-group."""
+    idx = sf_index(128)
+    return raw[..., idx].reshape(raw.shape[:-2] + (raw.shape[-2] * 128, 8))
+
+
+def gpu_quant_nvfp4(w: W.Workload, q, k, v):
+    p = sage.make_params(q, k, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                         smooth_q=w.smooth_q, bq=w.bq, bk=w.bk)
+    ws = sage.alloc_nvfp4_workspace(p)
+    qd, kd, vd = to_gpu(q, k, v)
+    view = sage.sage_quant_nvfp4(qd, kd, vd, p, ws)
+    torch.cuda.synchronize()
+    return p, ws, view, (qd, kd, vd)
+
+
+def gpu_attention_nvfp4(w: W.Workload, q, k, v):
+    p, ws, view, (qd, kd, vd) = gpu_quant_nvfp4(w, q, k, v)
+    o = torch.empty_like(qd)
+    sage.sage_attn_fwd_nvfp4_quantized(view, o, p)
+    torch.cuda.synchronize()
+    assert sage.sage_last_device_error() == 0
+    return p, ws, view, o
+
+
+def oracle_quant_nvfp4(w: W.Workload, q, k, v):
+    return oracle.quantize_nvfp4(q, k, v, bq=w.bq, smooth_k=w.smooth_k, smooth_q=w.smooth_q)
+
+
+def gpu_nvfp4_in_oracle_layout(view, p, ws) -> dict:
+    """The GPU's NVFP4 tensors rearranged to the oracle's layouts (codes one per
+    byte [.., N, d]; Q/K scales [.., N, d/16]; V scales [.., ceil(N/16), d])."""
+    t = {k: x.cpu().numpy() for k, x in sage.nvfp4_view_tensors(view, p, ws).items()}
+    N = p.N
+    Np = int(view.Np)
+    v4 = np.swapaxes(unpack_nibbles(t["v4t"]), 2, 3)             # [B,Hkv,Np,d]
+    T = Np // 128
+    sfv = np.empty(t["sfv"].shape[:2] + (T * 8, p.d), np.uint8)
+    idx = sf_index(128)                                            # [channel, grp]
+    for tt in range(T):
+        sfv[:, :, tt * 8:(tt + 1) * 8, :] = np.swapaxes(t["sfv"][:, :, tt][..., idx], 2, 3)
+    out = {
+        "q4": unpack_nibbles(t["q4"])[:, :, :N], "q4_pad": unpack_nibbles(t["q4"])[:, :, N:],
+        "sfq": unpack_sf(t["sfq"])[:, :, :N], "sfq_pad": unpack_sf(t["sfq"])[:, :, N:],
+        "k4": unpack_nibbles(t["k4"])[:, :, :N], "k4_pad": unpack_nibbles(t["k4"])[:, :, N:],
+        "sfk": unpack_sf(t["sfk"])[:, :, :N], "sfk_pad": unpack_sf(t["sfk"])[:, :, N:],
+        "v4": v4[:, :, :N], "v4_pad": v4[:, :, N:],
+        "sfv": sfv[:, :, :-(-N // 16)], "sfv_pad": sfv[:, :, -(-N // 16):],
+        "km": t["km"],
+    }
+    if "qbar" in t:
+        out["qbar"] = t["qbar"]
+        out["dS"] = t["dS"]
+    return out
+
+
+def compare_quant_nvfp4(w: W.Workload, g: dict, ref: dict) -> dict:
+    """Bit-exact comparison (codes, scales, km, qbar); delta_S within fp32 tolerance."""
+    bad = {}
+    for name in ("q4", "sfq", "k4", "sfk", "v4", "sfv", "km"):
+        a, b = np.asarray(g[name]), np.asarray(ref[name])
+        n = int(np.sum(a.view(np.uint32) != b.view(np.uint32))) if a.dtype.kind == "f" else int(np.sum(a != b))
+        if n:
+            bad[name] = n
+    for name in ("q4_pad", "sfq_pad", "k4_pad", "sfk_pad", "v4_pad", "sfv_pad"):
+        if np.any(g[name] != 0):
+            bad[name] = int(np.count_nonzero(g[name]))
+    if w.smooth_q:
+        if np.any(g["qbar"].view(np.uint32) != ref["qbar"].view(np.uint32)):
+            bad["qbar"] = 1
+        dS_g = g["dS"][..., :w.N].astype(np.float64)
+        dS_r = ref["dS"].astype(np.float64)
+        if np.abs(dS_g - dS_r).max() > 1e-5 * np.abs(dS_r).max() + 1e-6:
+            bad["dS"] = float(np.abs(dS_g - dS_r).max())
+    return bad
+
+
+def oracle_rows_nvfp4(w: W.Workload, quant, b, h, r0, r1):
+    return oracle.attention_nvfp4_head(quant, b, h, r0, r1, bq=w.bq, causal=w.causal, sm_scale=w.sm_scale)
