@@ -377,7 +377,9 @@ def main():
                        "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
                        "ms_step": e["ms_step"]}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        secs, ops_s, desc = oracle_sample(w, 8, 4, threads)
+        # about 10-15 s of CPU work on a 16-core host (all heads of batch 0,
+        # the 32 longest Q tiles of each)
+        secs, ops_s, desc = oracle_sample(w, min(32, w.Hkv), 32, threads)
         line["cpu_baseline"] = {"value": ops_s / secs / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
                                 "sample": desc, "seconds": secs}
     if rank == 0:
