@@ -151,17 +151,6 @@ sage_status make_maps(const sage_quant_view* v, const Dims& d, CUtensorMap* mQ, 
   return SAGE_OK;
 }
 
-// Scheduling of the two softmax warpgroups: taking turns (ping-pong) or running
-// concurrently.  SAGE_SOFTMAX_PINGPONG=0/1 overrides the per-mode default.
-int softmax_pingpong(int two_level) {
-  static const int env = [] {
-    const char* v = std::getenv("SAGE_SOFTMAX_PINGPONG");
-    return v ? std::atoi(v) : -1;
-  }();
-  (void)two_level;
-  return env >= 0 ? (env != 0) : 0;  // measured: concurrent is faster in both modes
-}
-
 AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d) {
   AttnArgs a{};
   a.B = (int)d.B;
@@ -184,7 +173,6 @@ AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d
   a.dS = p->smooth_q ? v->dS : nullptr;
   a.out_fp16 = p->dtype == SAGE_FP16;
   a.two_level = p->pv_accum == SAGE_PV_TWO_LEVEL;
-  a.pingpong = softmax_pingpong(a.two_level);
   return a;
 }
 

@@ -24,9 +24,11 @@
 //   WG2  softmax of Q tile 1
 //   WG3  level-2 accumulation O = alpha O + O_t for both tiles, and the epilogue
 // The two softmax warpgroups run concurrently (two softmax warps per SM
-// sub-partition hide each other's latencies); an optional ping-pong mode makes
-// them take turns on mbarriers.  TMEM (512 columns): S_i at [128 i, 128 i + 128)
-// and O_i at [256 + D i, 256 + D (i + 1)).  P goes through shared memory.
+// sub-partition hide each other's latencies).  TMEM (512 columns): S_i at
+// [128 i, 128 i + 128), holding the magic fill 0x4B400000 between uses (QK^T
+// accumulates onto it, see below), and O_i at [256 + D i, 256 + D (i + 1)).
+// P goes through shared memory, two buffers per tile, so the softmax of tile
+// j + 1 never waits for P V(j).
 // Two P~V accumulation modes (template TWO_LEVEL):
 //   two-level: PV(i, j) writes a fresh O_t into S_i's columns (S is dead once
 //     the softmax read it); the correction warpgroup adds it into O_i on CUDA
@@ -34,6 +36,8 @@
 //   TMEM accumulator: PV(i, j) accumulates into O_i itself (tcgen05 keeps the
 //     FP8 products' sum in full FP32); before it, the correction warpgroup
 //     rescales the rows of O_i whose max grew (alpha != 1; alpha == 1 is exact).
+#include <cfloat>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -58,15 +62,17 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 template <int D>
 struct Smem {
-  static constexpr uint32_t kQ = 128 * D, kK = 128 * D, kV = D * 128, kP = 128 * 128;
+  static constexpr uint32_t kQ = 128 * D, kK = 128 * D, kV = D * 128, kP = 128 * 128;  // kP: one P buffer
   static constexpr uint32_t oQ = 0;                      // 2 tiles
   static constexpr uint32_t oK = oQ + 2 * kQ;            // kStages
   static constexpr uint32_t oV = oK + kStages * kK;      // kStages
-  static constexpr uint32_t oP = oV + kStages * kV;      // 2 tiles
-  static constexpr uint32_t oAlpha = oP + 2 * kP;        // float[2][128]
-  static constexpr uint32_t oL = oAlpha + 2 * 128 * 4;   // float[2][128]
+  static constexpr uint32_t oP = oV + kStages * kV;      // [tile][2 buffers]
+  static constexpr uint32_t kDS = 2 * 2 * 128 * 4;      // delta_S rows of one key tile
+  static constexpr uint32_t oDS = oP + 4 * kP;           // kStages
+  static constexpr uint32_t oAlpha = oDS + kStages * kDS;  // float[tile][buffer][128]
+  static constexpr uint32_t oL = oAlpha + 4 * 128 * 4;   // float[2][128]
   static constexpr uint32_t oBar = oL + 2 * 128 * 4;
-  static constexpr uint32_t kNumBars = 1 + 3 * kStages + 7 * 2 + 1;
+  static constexpr uint32_t kNumBars = 1 + 3 * kStages + 2 + 4 + 4 + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = oTmem + 16 + 1024;  // + alignment slack
 };
@@ -86,17 +92,19 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
 
 struct Bars {
   uint64_t* q_full;
-  uint64_t* k_full;    // [kStages]
+  uint64_t* k_full;    // [kStages]  K_j (+ delta_S rows) landed
   uint64_t* v_full;    // [kStages]
   uint64_t* kv_empty;  // [kStages]
   uint64_t* s_full;    // [2]  QK^T of tile i done            (tcgen05.commit)
-  uint64_t* p_full;    // [2]  P_i and alpha_i written         (128 softmax threads)
-  uint64_t* ot_full;   // [2]  O_t of tile i done              (tcgen05.commit)
-  uint64_t* r_free;    // [2]  S_i columns free for the next QK^T (two-level: correction
-                       //      consumed O_t_i; TMEM accumulator: softmax read S_i)
-  uint64_t* turn;      // [2]  softmax ping-pong: tile i may run (128 threads of the other tile)
-  uint64_t* l_ready;   // [2]  final l of tile i in shared memory
-  uint64_t* o_ready;   // [2]  (TMEM accumulator mode) O_i rescaled for the next P V
+  uint64_t* p_full;    // [tile][buffer j & 1]  P_i(j) and alpha_i(j) written (one arrival per softmax
+                       //      warp); one barrier per buffer keeps every waiter at most one phase behind
+  uint64_t* p_empty;   // [tile][buffer]  the P V that read that P buffer retired (tcgen05.commit)
+  uint64_t* ot_full;   // [2]  P V of tile i retired              (tcgen05.commit)
+  uint64_t* r_free;    // [2]  S_i columns hold the magic fill again and may take the next QK^T
+                       //      (TMEM accumulator: the softmax refilled them; two-level: the
+                       //      correction consumed O_t_i and refilled them); one arrival per warp
+  uint64_t* l_ready;   // [2]  final l of tile i in shared memory (128 threads)
+  uint64_t* o_ready;   // [2]  (TMEM accumulator mode) O_i rescaled for the next P V (one per warp)
   uint64_t* mma_done;  // all tensor-core work of the CTA retired (one commit at the end)
 };
 
@@ -117,6 +125,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* sK = smem + L::oK;
   uint8_t* sV = smem + L::oV;
   uint8_t* sP = smem + L::oP;
+  const float* sDS = reinterpret_cast<const float*>(smem + L::oDS);
   float* s_alpha = reinterpret_cast<float*>(smem + L::oAlpha);
   float* s_l = reinterpret_cast<float*>(smem + L::oL);
   uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L::oBar);
@@ -127,10 +136,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   bar.kv_empty = bar.v_full + kStages;
   bar.s_full = bar.kv_empty + kStages;
   bar.p_full = bar.s_full + 2;
-  bar.ot_full = bar.p_full + 2;
+  bar.p_empty = bar.p_full + 4;
+  bar.ot_full = bar.p_empty + 4;
   bar.r_free = bar.ot_full + 2;
-  bar.turn = bar.r_free + 2;
-  bar.l_ready = bar.turn + 2;
+  bar.l_ready = bar.r_free + 2;
   bar.o_ready = bar.l_ready + 2;
   bar.mma_done = bar.o_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oTmem);
@@ -162,12 +171,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar.s_full[i], 1);
-      mbar_init(&bar.p_full[i], 128);
       mbar_init(&bar.ot_full[i], 1);
-      mbar_init(&bar.r_free[i], 128);
-      mbar_init(&bar.turn[i], 128);
+      mbar_init(&bar.r_free[i], 4);
       mbar_init(&bar.l_ready[i], 128);
-      mbar_init(&bar.o_ready[i], 128);
+      mbar_init(&bar.o_ready[i], 4);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bar.p_full[i], 4);
+      mbar_init(&bar.p_empty[i], 1);
     }
     mbar_init(bar.mma_done, 1);
     mbar_fence_init();
@@ -180,6 +191,18 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // S accumulators start at the int32 bit pattern of 1.5 * 2^23: QK^T accumulates
+  // onto it, so TMEM returns 0x4B400000 + acc, which read as fp32 is exactly
+  // 12582912 + acc (|acc| <= 127 * 127 * 128 < 2^22): no int -> float step.
+  if (wg == 1 || wg == 2) {
+    const uint32_t tS0 = tmem + 128 * (wg - 1) + ((uint32_t)((warp & 3) * 32) << 16);
+#pragma unroll
+    for (int c = 0; c < 128; c += 8) tmem_fill8(tS0 + c, kMagicBits);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (wg == 0) {
     regs_dec<kRegsProducer>();
@@ -191,6 +214,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
       const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np);
       const int vrow = (b * a.Hkv + g) * D;
+      const int ds_rows = kTile / a.bq;  // Q blocks per tile (1 or 2)
+      const uint32_t ds_bytes = (uint32_t)((nTi[0] > 0) + (nTi[1] > 0)) * ds_rows * 512;
       mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
       for (int i = 0; i < 2; ++i)
         if (nTi[i] > 0) tma_load_2d(sQ + i * L::kQ, &tmQ, bar.q_full, 0, (int)(qhead + (int64_t)(2 * pr + i) * kTile));
@@ -200,8 +225,19 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         const int s = j % kStages;
         if (j >= kStages) ok = mbar_wait(&bar.kv_empty[s], ((j / kStages) + 1) & 1);
         if (!ok) break;
-        mbar_expect_tx(&bar.k_full[s], L::kK);
+        mbar_expect_tx(&bar.k_full[s], L::kK + (HAS_DS ? ds_bytes : 0u));
         tma_load_2d(sK + s * L::kK, &tmK, &bar.k_full[s], 0, krow0 + j * kTile);
+        if (HAS_DS) {
+          // delta_S[b, h, Q block, keys of tile j] for the Q blocks of both tiles
+          for (int i = 0; i < 2; ++i)
+            for (int hb = 0; hb < ds_rows; ++hb)
+              if (nTi[i] > 0) {
+                const int blk = min((2 * pr + i) * ds_rows + hb, a.Tm - 1);
+                bulk_load_1d(smem + L::oDS + s * L::kDS + (i * 2 + hb) * 512,
+                             a.dS + ((int64_t)(b * a.Hq + h) * a.Tm + blk) * a.Np + (int64_t)j * kTile, 512,
+                             &bar.k_full[s]);
+              }
+        }
         mbar_expect_tx(&bar.v_full[s], L::kV);
         tma_load_2d(sV + s * L::kV, &tmV, &bar.v_full[s], j * kTile, vrow);
       }
@@ -222,12 +258,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
             mma_i8(tmem + 128 * i, make_sdesc(aQ + kk * 32, kSboQK, kSwzQK), make_sdesc(aK + kk * 32, kSboQK, kSwzQK),
-                   kIdescQK, kk > 0 ? 1u : 0u);
+                   kIdescQK, 1u);  // accumulate onto the magic fill
           mma_commit(&bar.s_full[i]);
         };
         auto issue_pv = [&](int i, int j) {
           const int s = j % kStages;
-          const uint32_t aP = aP0 + i * L::kP, aV = smem_u32(sV + s * L::kV);
+          const uint32_t aP = aP0 + (i * 2 + (j & 1)) * L::kP, aV = smem_u32(sV + s * L::kV);
           // two-level: a fresh O_t tile in S_i's columns; else accumulate into O_i
           const uint32_t dst = TWO_LEVEL ? tmem + 128 * i : tmem + 256 + D * i;
 #pragma unroll
@@ -235,10 +271,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             mma_f8f6f4(dst, make_sdesc(aP + kk * 32, 1024, kSwizzle128B), make_sdesc(aV + kk * 32, 1024, kSwizzle128B),
                        kIdescPV, (kk > 0 || (!TWO_LEVEL && j > 0)) ? 1u : 0u);
           mma_commit(&bar.ot_full[i]);
+          mma_commit(&bar.p_empty[i * 2 + (j & 1)]);
         };
         // Two independent per-tile chains, each op issued as soon as its inputs
         // are ready (non-blocking polls), so one tile never holds the other back.
-        //   QK(i,j): K_j landed; j > 0: S_i columns free (r_free) and, two-level,
+        //   QK(i,j): K_j landed; j > 0: S_i columns refilled (r_free) and, two-level,
         //            PV(i,j-1) issued (its O_t shares those columns)
         //   PV(i,j): QK(i,j) issued; V_j landed; P_i(j) written; TMEM-accumulator
         //            mode, j > 0: O_i rescaled (o_ready)
@@ -259,7 +296,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
               next_qk[i] = jq + 1;
               progress = true;
             }
-            if (jp < nTi[i] && next_qk[i] > jp && mbar_test_wait(smem_u32(&bar.p_full[i]), jp & 1) &&
+            if (jp < nTi[i] && next_qk[i] > jp &&
+                mbar_test_wait(smem_u32(&bar.p_full[i * 2 + (jp & 1)]), (jp >> 1) & 1) &&
                 mbar_test_wait(smem_u32(&bar.v_full[jp % kStages]), (jp / kStages) & 1) &&
                 (TWO_LEVEL || jp == 0 || mbar_test_wait(smem_u32(&bar.o_ready[i]), (jp - 1) & 1))) {
               tc_fence_after();
@@ -274,16 +312,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             ++released;
           }
           if (next_pv[0] >= nTi[0] && next_pv[1] >= nTi[1] && released >= nT) break;
+          // spin (a sleep here delays the reaction to a ready operand), bounded by the idle time
           if (progress) {
             t_idle = 0;
           } else if (t_idle == 0) {
-            __nanosleep(32);
             t_idle = globaltimer_ns();
           } else if (globaltimer_ns() - t_idle > g_wait_limit_ns) {
             record_error(kDevErrTimeout);
             ok = false;
-          } else {
-            __nanosleep(32);
           }
         }
         // every tensor-core op retired before TMEM is released
@@ -304,56 +340,62 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const int qblk = min((int)(qrow / a.bq), a.Tm - 1);
     const float row_scale = a.s_q[(int64_t)(b * a.Hq + h) * a.Tm + qblk] * a.scale_log2;
     const float* sk = a.s_k + (int64_t)(b * a.Hkv + g) * a.Tn;
-    const float* dsr = HAS_DS ? a.dS + ((int64_t)(b * a.Hq + h) * a.Tm + qblk) * a.Np : nullptr;
-    uint8_t* myP = sP + ti * L::kP + row * 128;
+    const int ds_half = (a.bq == 64 && row >= 64) ? 1 : 0;  // warp-uniform
+    float sk_lo = __ldg(sk + 0), sk_hi = __ldg(sk + min(64 / a.bk, a.Tn - 1));
+    const float sl2 = a.scale_log2;
+    const float2 neg_magic = make_float2(-kMagic, -kMagic);
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
 
-    for (int j = 0; j < nT && ok; ++j) {
-      // ping-pong: tile 0 runs iteration j after tile 1 finished j-1; tile 1 after tile 0 finished j
-      if (a.pingpong && ti == 0 && j > 0) ok = mbar_wait_warp(&bar.turn[0], (j - 1) & 1);
-      if (a.pingpong && ti == 1) ok = ok && mbar_wait_warp(&bar.turn[1], j & 1);
-      if (!ok) break;
-      if (j < nTi[ti]) {
-        if (!(ok = mbar_wait_warp(&bar.s_full[ti], j & 1))) break;
-        tc_fence_after();
-        uint32_t s[128];
-        tmem_ld32p(tS + 0, s + 0);
-        tmem_ld32p(tS + 32, s + 32);
-        tmem_ld32p(tS + 64, s + 64);
-        tmem_ld32p(tS + 96, s + 96);
-        const int col0 = j * kTile;
-        const float a_lo = row_scale * __ldg(sk + min(col0 / a.bk, a.Tn - 1));
-        const float a_hi = row_scale * __ldg(sk + min((col0 + 64) / a.bk, a.Tn - 1));
-        tmem_ld_wait();
-        if (!TWO_LEVEL) {  // S_i is in registers: the next QK^T may overwrite its columns
-          tc_fence_before();
-          mbar_arrive(&bar.r_free[ti]);
-        }
-        // t = float(acc) * a (+ delta_S * sm_scale * log2 e), in place (as float bits)
+    for (int j = 0; j < nTi[ti] && ok; ++j) {
+      if (!(ok = mbar_wait_warp(&bar.s_full[ti], j & 1))) break;
+      tc_fence_after();
+      uint32_t s[128];  // fp32 bits of y = 12582912 + acc (acc = the INT8 dot product)
+      tmem_ld32p(tS + 0, s + 0);
+      tmem_ld32p(tS + 32, s + 32);
+      tmem_ld32p(tS + 64, s + 64);
+      tmem_ld32p(tS + 96, s + 96);
+      const int col0 = j * kTile;
+      // a = s_q s_k sm_scale log2 e per 64-key half, kept > 0 so that a masked
+      // -inf stays -inf (a zero scale only multiplies zero dot products)
+      const float a_lo = fmaxf(row_scale * sk_lo, FLT_MIN), a_hi = fmaxf(row_scale * sk_hi, FLT_MIN);
+      // next tile's key-block scales (their load latency hides behind this tile)
+      sk_lo = __ldg(sk + min((col0 + kTile) / a.bk, a.Tn - 1));
+      sk_hi = __ldg(sk + min((col0 + kTile + 64) / a.bk, a.Tn - 1));
+      const float* dsr = sDS + (j % kStages) * (L::kDS / 4) + (ti * 2 + ds_half) * 128;
+      if (HAS_DS && !(ok = mbar_wait_warp(&bar.k_full[j % kStages], (j / kStages) & 1))) break;
+      tmem_ld_wait();
+      if (!TWO_LEVEL) {
+        // S_i is in registers: restore the magic fill, then the next QK^T may run
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) tmem_fill8(tS + c, kMagicBits);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.r_free[ti]);
+      }
+      const bool need_mask = (col0 + kTile > a.N) || (CAUSAL && j == qtile);
+      float mx;
+      if (HAS_DS) {
+        // t = (y - 12582912) a + delta_S sm_scale log2 e, in place
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
           const float sc = c < 64 ? a_lo : a_hi;
-          float2 x = make_float2(magic_bits_to_float(s[c]), magic_bits_to_float(s[c + 1]));
-          x = fadd2(x, make_float2(-kMagic, -kMagic));  // exact
-          float2 t;
-          if (HAS_DS) {
-            const float2 ds = __ldg(reinterpret_cast<const float2*>(dsr + col0 + c));
-            t = ffma2(x, make_float2(sc, sc), fmul2(ds, make_float2(a.scale_log2, a.scale_log2)));
-          } else {
-            t = fmul2(x, make_float2(sc, sc));
-          }
+          const float2 x = fadd2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), neg_magic);
+          const float2 ds = *reinterpret_cast<const float2*>(dsr + c);
+          const float2 t = ffma2(x, make_float2(sc, sc), fmul2(ds, make_float2(sl2, sl2)));
           s[c] = __float_as_uint(t.x);
           s[c + 1] = __float_as_uint(t.y);
         }
-        const bool need_mask = (col0 + kTile > a.N) || (CAUSAL && j == qtile);
-        if (need_mask) {
+      }
+      if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int col = col0 + c;
-            if (col >= a.N || (CAUSAL && col > qrow)) s[c] = __float_as_uint(-INFINITY);
-          }
+        for (int c = 0; c < 128; ++c) {
+          const int col = col0 + c;
+          if (col >= a.N || (CAUSAL && col > qrow)) s[c] = __float_as_uint(-INFINITY);
         }
+      }
+      if (HAS_DS) {
         // row max: 8 independent 3-input chains, then a short tree (max is exact)
         float mx8[8];
 #pragma unroll
@@ -363,46 +405,69 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mx8[k] = fmax3(mx8[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        const float m_new = fmaxf(m, mx);
-        const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
-        const float mm = (m_new == -INFINITY) ? 0.0f : m_new - kLog2_448;
-        // TMEM-accumulator mode: PV(j-1) must have read P_i before it is rewritten
-        // (two-level: guaranteed by the chain O_t -> correction -> next QK^T)
-        if (!TWO_LEVEL && j > 0 && !(ok = mbar_wait_warp(&bar.ot_full[ti], (j - 1) & 1))) break;
-        // P = exp2(t - m + log2 448) -> E4M3 -> shared memory (128B-swizzled K-major)
-        // row sum: 8 independent f32x2 partial sums (fp32 rounding order only)
-        float2 rs[8];
+        mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+      } else {
+        // y is monotonic in acc: take the max of each 64-key half on y and scale
+        // only the two maxima
+        float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) rs[k] = make_float2(0.0f, 0.0f);
+        for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-        for (int grp = 0; grp < 8; ++grp) {
-          uint32_t w[4];
+        for (int c = 0; c < 64; c += 8)
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const int c = grp * 16 + e;
-            const float2 u0 = fadd2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
-                                    make_float2(-mm, -mm));
-            const float2 u1 = fadd2(make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])),
-                                    make_float2(-mm, -mm));
-            const float2 p0 = make_float2(ex2_approx(u0.x), ex2_approx(u0.y));
-            const float2 p1 = make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
-            rs[e / 2] = fadd2(rs[e / 2], p0);
-            rs[e / 2 + 1] = fadd2(rs[e / 2 + 1], p1);
-            w[e / 4] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
+          for (int k = 0; k < 4; ++k) {
+            mx8[k] = fmax3(mx8[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
+            mx8[4 + k] = fmax3(mx8[4 + k], __uint_as_float(s[64 + c + 2 * k]), __uint_as_float(s[64 + c + 2 * k + 1]));
           }
-          *reinterpret_cast<uint4*>(myP + ((grp ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        const float2 rs2 = fadd2(fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3])),
-                                 fadd2(fadd2(rs[4], rs[5]), fadd2(rs[6], rs[7])));
-        s_alpha[ti * 128 + row] = alpha;
-        tc_fence_before();
-        fence_proxy_async_smem();
-        mbar_arrive(&bar.p_full[ti]);
-        l = fmaf(l, alpha, rs2.x + rs2.y);
-        m = m_new;
+        const float ylo = fmax3(mx8[0], mx8[1], fmaxf(mx8[2], mx8[3]));
+        const float yhi = fmax3(mx8[4], mx8[5], fmaxf(mx8[6], mx8[7]));
+        mx = fmaxf((ylo - kMagic) * a_lo, (yhi - kMagic) * a_hi);
       }
-      if (a.pingpong) mbar_arrive(&bar.turn[ti ^ 1]);
+      const float m_new = fmaxf(m, mx);
+      const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
+      const float mm = (m_new == -INFINITY) ? 0.0f : m_new - kLog2_448;
+      // P buffer (j & 1) is free once P V(j - 2) retired
+      if (j >= 2 && !(ok = mbar_wait_warp(&bar.p_empty[ti * 2 + (j & 1)], ((j >> 1) - 1) & 1))) break;
+      uint8_t* myP = sP + (ti * 2 + (j & 1)) * L::kP + row * 128;
+      // P = exp2(t - m + log2 448) -> E4M3 -> shared memory (128B-swizzled K-major)
+      // row sum: 8 independent f32x2 partial sums (fp32 rounding order only)
+      float2 rs[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) rs[k] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int grp = 0; grp < 8; ++grp) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const int c = grp * 16 + e;
+          float2 u0, u1;
+          const float2 y0 = make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          const float2 y1 = make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+          if (HAS_DS) {
+            u0 = fadd2(y0, make_float2(-mm, -mm));
+            u1 = fadd2(y1, make_float2(-mm, -mm));
+          } else {
+            const float sc = c < 64 ? a_lo : a_hi;
+            u0 = ffma2(fadd2(y0, neg_magic), make_float2(sc, sc), make_float2(-mm, -mm));
+            u1 = ffma2(fadd2(y1, neg_magic), make_float2(sc, sc), make_float2(-mm, -mm));
+          }
+          const float2 p0 = make_float2(ex2_approx(u0.x), ex2_approx(u0.y));
+          const float2 p1 = make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
+          rs[e / 2] = fadd2(rs[e / 2], p0);
+          rs[e / 2 + 1] = fadd2(rs[e / 2 + 1], p1);
+          w[e / 4] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
+        }
+        *reinterpret_cast<uint4*>(myP + ((grp ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      const float2 rs2 = fadd2(fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3])),
+                               fadd2(fadd2(rs[4], rs[5]), fadd2(rs[6], rs[7])));
+      s_alpha[(ti * 2 + (j & 1)) * 128 + row] = alpha;
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.p_full[ti * 2 + (j & 1)]);
+      l = fmaf(l, alpha, rs2.x + rs2.y);
+      m = m_new;
     }
     s_l[ti * 128 + row] = l;
     mbar_arrive(&bar.l_ready[ti]);
@@ -414,14 +479,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
     uint32_t x[32], y[32];
+    // every phase of p_full[tile][buffer] is waited in order, j = 0 included (a
+    // parity wait on a phase two ahead of the barrier would pass at once)
     if constexpr (TWO_LEVEL) {
       for (int j = 0; j < nT && ok; ++j) {
         for (int i = 0; i < 2; ++i) {
           if (j >= nTi[i]) continue;
           if (!(ok = mbar_wait_warp(&bar.ot_full[i], j & 1))) break;
-          if (!(ok = mbar_wait_warp(&bar.p_full[i], j & 1))) break;
+          if (!(ok = mbar_wait_warp(&bar.p_full[i * 2 + (j & 1)], (j >> 1) & 1))) break;
           tc_fence_after();
-          const float alpha = s_alpha[i * 128 + row];
+          const float alpha = s_alpha[(i * 2 + (j & 1)) * 128 + row];
           const uint32_t tOt = tmem + 128 * i + lane_off, tO = tmem + 256 + D * i + lane_off;
           if (j == 0) {
   #pragma unroll
@@ -462,25 +529,28 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
               if (c + 16 < D) tmem_ld_wait();
             }
           }
+          // S_i's columns get the magic fill back (O_t covered the first D of them;
+          // the softmax read all 128 before P V(j) could run)
+  #pragma unroll
+          for (int c = 0; c < 128; c += 8) tmem_fill8(tOt + c, kMagicBits);
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&bar.r_free[i]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.r_free[i]);
         }
       }
     } else {
       // O_i accumulates in TMEM; before PV(i, j) adds tile j, rows whose max grew
       // are rescaled by alpha = e^(m_old - m_new).  A warp whose 32 rows all have
       // alpha == 1 leaves O_i untouched (exact).
-      // (every phase of p_full is waited in order, j = 0 included: a parity wait
-      // on a phase two ahead of the barrier would pass at once)
       for (int j = 0; j < nT && ok; ++j) {
         for (int i = 0; i < 2; ++i) {
           if (j >= nTi[i]) continue;
-          if (!(ok = mbar_wait_warp(&bar.p_full[i], j & 1))) break;
+          if (!(ok = mbar_wait_warp(&bar.p_full[i * 2 + (j & 1)], (j >> 1) & 1))) break;
           if (j == 0) continue;
           if (!(ok = mbar_wait_warp(&bar.ot_full[i], (j - 1) & 1))) break;
           tc_fence_after();
-          const float alpha = s_alpha[i * 128 + row];
+          const float alpha = s_alpha[(i * 2 + (j & 1)) * 128 + row];
           if (__any_sync(0xffffffffu, alpha != 1.0f)) {
             const uint32_t tO = tmem + 256 + D * i + lane_off;
 #pragma unroll
@@ -499,7 +569,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             tmem_st_wait();
           }
           tc_fence_before();
-          mbar_arrive(&bar.o_ready[i]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.o_ready[i]);
         }
       }
     }

@@ -54,7 +54,6 @@ struct AttnArgs {
   void* o;          // [B,Hq,N,D] bf16/fp16
   int out_fp16;
   int two_level;  // 1: fresh O_t per key tile + FP32 add on CUDA cores; 0: TMEM FP32 accumulator
-  int pingpong;   // 1: the two softmax warpgroups take turns; 0: they run concurrently
   // NVFP4 scale blocks (1 KB per 128-row tile)
   const uint8_t* sfq;
   const uint8_t* sfk;
