@@ -10,8 +10,10 @@
 // Bit-exactness with the plain definitions: column sums are accumulated in
 // fp64 (the partial sums of bf16/fp16 inputs are exact, so the order does
 // not matter), divided in fp64 and rounded once to fp32; every division of
-// the quantisers is an IEEE fp32 division (__fdiv_rn) and the INT8 rounding
-// is round-half-to-even (__float2int_rn).  Do not build with fast-math.
+// the quantisers is an IEEE fp32 division (__fdiv_rn) -- per element it is
+// replaced by a multiplication with the reciprocal wherever that provably
+// gives the same code (quant_i8 / quant_e4m3x2 below) -- and the INT8 rounding
+// is round-half-to-even.  Do not build with fast-math.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -61,11 +63,52 @@ __device__ __forceinline__ int rows_valid(int N, int64_t r0, int rows) {
   return v <= 0 ? 0 : (v < rows ? (int)v : rows);
 }
 
-__device__ __forceinline__ int8_t quant_i8(float x, float s) {
+// Codes of a quotient x / s without a division per element.  With r = RN(1/s),
+// y = RN(x r) is within 1.5 ulp of RN(x / s) (the quotient the definition
+// rounds).  Every code conversion is monotonic, so when y (1 - 2^-21) and
+// y (1 + 2^-21) -- a bracket of at least +-3.5 ulp around y -- get the same code,
+// RN(x / s) gets it too; otherwise (within ~4 ulp of a rounding boundary, about
+// one value in 10^5) the exact quotient __fdiv_rn(x, s) decides.  Subnormal y
+// only arise for codes that are 0 either way.
+constexpr float kBracketLo = 1.0f - 0x1p-21f, kBracketHi = 1.0f + 0x1p-21f;
+
+// rint for |v| < 2^22 in one rounding: the fp32 bits of v + 1.5 * 2^23 (RNE)
+__device__ __forceinline__ int rint_bits(float v) { return __float_as_int(__fadd_rn(v, 12582912.0f)); }
+
+__device__ __forceinline__ int8_t quant_i8(float x, float s, float r) {
   if (s == 0.0f) return 0;
-  int q = __float2int_rn(__fdiv_rn(x, s));
+  const float y = __fmul_rn(x, r);
+  const int lo = __float_as_int(__fmaf_rn(y, kBracketLo, 12582912.0f));
+  const int hi = __float_as_int(__fmaf_rn(y, kBracketHi, 12582912.0f));
+  int q = (lo == hi) ? lo - 0x4B400000 : __float2int_rn(__fdiv_rn(x, s));
   q = q > 127 ? 127 : (q < -127 ? -127 : q);
   return static_cast<int8_t>(q);
+}
+
+// Two E4M3 codes of x0 / s, x1 / s (lo byte x0); s > 0, r = RN(1/s).
+__device__ __forceinline__ uint32_t quant_e4m3x2(float x0, float x1, float s, float r) {
+  const float y0 = __fmul_rn(x0, r), y1 = __fmul_rn(x1, r);
+  const uint32_t lo = cvt_e4m3x2(__fmul_rn(y0, kBracketLo), __fmul_rn(y1, kBracketLo));
+  const uint32_t hi = cvt_e4m3x2(__fmul_rn(y0, kBracketHi), __fmul_rn(y1, kBracketHi));
+  return lo == hi ? lo : cvt_e4m3x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
+}
+
+// Eight E2M1 codes of x[e] / s (element e in bits 4e..4e+3); s > 0, r = RN(1/s).
+__device__ __forceinline__ uint32_t quant_e2m1x8(const float (&x)[8], float s, float r) {
+  float l[8], h[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float y = __fmul_rn(x[e], r);
+    l[e] = __fmul_rn(y, kBracketLo);
+    h[e] = __fmul_rn(y, kBracketHi);
+  }
+  const uint32_t lo = cvt_e2m1x8(l[0], l[1], l[2], l[3], l[4], l[5], l[6], l[7]);
+  const uint32_t hi = cvt_e2m1x8(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]);
+  if (lo == hi) return lo;
+  float q[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) q[e] = __fdiv_rn(x[e], s);
+  return cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
 }
 
 __device__ __forceinline__ uint2 pack8_i8(const int8_t (&c)[8]) {
@@ -219,10 +262,11 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const __grid_constan
     if (threadIdx.x == 0) s_bmax[kb] = m;
   }
   __syncthreads();
-  float sk[NKB];
+  float sk[NKB], rk[NKB];
 #pragma unroll
   for (int kb = 0; kb < NKB; ++kb) {
     sk[kb] = __fdiv_rn(s_bmax[kb], 127.0f);
+    rk[kb] = sk[kb] == 0.0f ? 0.0f : __frcp_rn(sk[kb]);
     const int gb = tile * NKB + kb;
     if (threadIdx.x == 0 && gb < a.Tn) a.s_k[(int64_t)bg * a.Tn + gb] = sk[kb];
   }
@@ -232,7 +276,7 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const __grid_constan
     const int r = rg + p * RG;
     int8_t c8[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], sk[p / PPB]) : (int8_t)0;
+    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], sk[p / PPB], rk[p / PPB]) : (int8_t)0;
     *reinterpret_cast<uint2*>(k8 + (r0 + r) * D + ch * 8) = pack8_i8(c8);
   }
 
@@ -242,6 +286,7 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const __grid_constan
     constexpr int RUNS = kTile / 16 / TG;      // 16-token runs per thread
     const int c = threadIdx.x % D, tg = threadIdx.x / D;
     const float sv = s_sv[c];
+    const float rv = sv == 0.0f ? 0.0f : __frcp_rn(sv);
 #pragma unroll
     for (int q = 0; q < RUNS; ++q) {
       const int run = tg * RUNS + q;
@@ -250,11 +295,8 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const __grid_constan
       for (int u = 0; u < 16; u += 4) {
         float f[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float v = to_float(sV[(run * 16 + u + e) * SL::kPitch + c]);
-          f[e] = (sv == 0.0f) ? 0.0f : __fdiv_rn(v, sv);
-        }
-        w[u / 4] = cvt_e4m3x2(f[0], f[1]) | (cvt_e4m3x2(f[2], f[3]) << 16);
+        for (int e = 0; e < 4; ++e) f[e] = to_float(sV[(run * 16 + u + e) * SL::kPitch + c]);
+        w[u / 4] = sv == 0.0f ? 0u : quant_e4m3x2(f[0], f[1], sv, rv) | (quant_e4m3x2(f[2], f[3], sv, rv) << 16);
       }
       *reinterpret_cast<uint4*>(sVt + c * kTile + ((run ^ (c & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
@@ -333,13 +375,14 @@ __global__ void __launch_bounds__(kThreads) q_quant_kernel(QuantArgs a) {
       for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x[p][e]));
   const float amax = block_max_nonneg(am, s_red);
   const float s = __fdiv_rn(amax, 127.0f);
+  const float rq = s == 0.0f ? 0.0f : __frcp_rn(s);
   if (threadIdx.x == 0) a.s_q[(int64_t)bh * a.Tm + blk] = s;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int r = rg + p * RG;
     int8_t c8[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], s) : (int8_t)0;
+    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], s, rq) : (int8_t)0;
     *reinterpret_cast<uint2*>(q8 + (r0 + r) * D + ch * 8) = pack8_i8(c8);
   }
 }
@@ -347,51 +390,79 @@ __global__ void __launch_bounds__(kThreads) q_quant_kernel(QuantArgs a) {
 // ---------------------------------------------------------------------------
 // Pass 3 (smooth Q): delta_S[b,h,i,j] = sum_c qbar[i,c] * gamma(K)[j,c] for one
 // 128-key tile and every Q block i.  fp32 accumulation in channel order.
-// grid (Np/128, B*Hq); dynamic smem: D*128 floats (gamma^T)
+// gamma(K)^T [D][128] and 32-block chunks of qbar^T [D][32] sit in shared
+// memory; each thread accumulates a 4-block x 4-key tile (two f32x2 FMAs per
+// block and channel), so every shared load feeds eight FMAs.
+// grid (Np/128, B*Hq), 256 threads; dynamic smem: (D*128 + D*32) floats
+constexpr int kDsBlocks = 32;  // Q blocks per chunk
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) delta_s_kernel(QuantArgs a) {
-  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG;
-  extern __shared__ float s_gT[];  // [D][kTile]
+  extern __shared__ float s_ds[];
+  float* s_gT = s_ds;               // [D][kTile]
+  float* s_qT = s_ds + D * kTile;   // [D][kDsBlocks]
   const int bh = blockIdx.y, tile = blockIdx.x;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const int bg = b * a.Hkv + h / (a.Hq / a.Hkv);
   const int64_t r0 = (int64_t)tile * kTile;
   const int valid = rows_valid(a.N, r0, kTile);
-  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
   const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
   const float* km = a.km + (int64_t)bg * D;
+  // gamma(K) -> shared, transposed.  A warp takes 16 rows x 2 adjacent 8-channel
+  // chunks per step: 32-byte row segments from global, and its transposed
+  // stores hit each bank at most twice.
+  {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
-    float x[8];
-    if (r < valid) {
-      load8<T>(K + (r0 + r) * D + ch * 8, x);
+    for (int it = 0; it < (kTile / 16) * (D / 16) / (kThreads / 32); ++it) {
+      const int item = warp + it * (kThreads / 32);
+      const int r = (item % (kTile / 16)) * 16 + lane / 2;
+      const int chunk = (item / (kTile / 16)) * 2 + (lane & 1);
+      float x[8];
+      if (r < valid) {
+        load8<T>(K + (r0 + r) * D + chunk * 8, x);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], km[ch * 8 + e]);
-    } else {
+        for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], km[chunk * 8 + e]);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+        for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_gT[(chunk * 8 + e) * kTile + r] = x[e];
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s_gT[(ch * 8 + e) * kTile + r] = x[e];
   }
-  __syncthreads();
-  const int key = threadIdx.x % kTile;
+  const int kg = threadIdx.x % 32, bgp = threadIdx.x / 32;  // keys 4 kg.., blocks 4 bgp..
   const float* qb = a.qbar + (int64_t)bh * a.Tm * D;
-  float* out = a.dS + (int64_t)bh * a.Tm * a.Np + r0 + key;
-  for (int i0 = threadIdx.x / kTile; i0 < a.Tm; i0 += 2 * (kThreads / kTile)) {
-    const int i1 = i0 + kThreads / kTile;
-    float acc0 = 0.0f, acc1 = 0.0f;
-    const float* q0 = qb + (int64_t)i0 * D;
-    const float* q1 = qb + (int64_t)min(i1, a.Tm - 1) * D;
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) {
-      const float gv = s_gT[c * kTile + key];
-      acc0 = fmaf(__ldg(q0 + c), gv, acc0);
-      acc1 = fmaf(__ldg(q1 + c), gv, acc1);
+  float* out = a.dS + (int64_t)bh * a.Tm * a.Np + r0 + 4 * kg;
+  for (int i0 = 0; i0 < a.Tm; i0 += kDsBlocks) {
+    __syncthreads();  // gamma^T written / previous chunk consumed
+    for (int idx = threadIdx.x; idx < kDsBlocks * D; idx += kThreads) {
+      const int blk = idx % kDsBlocks, c = idx / kDsBlocks;  // conflict-free stores
+      s_qT[c * kDsBlocks + blk] = (i0 + blk < a.Tm) ? qb[(int64_t)(i0 + blk) * D + c] : 0.0f;
     }
-    out[(int64_t)i0 * a.Np] = acc0;
-    if (i1 < a.Tm) out[(int64_t)i1 * a.Np] = acc1;
+    __syncthreads();
+    float2 acc[4][2];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = make_float2(0.0f, 0.0f);
+#pragma unroll 4
+    for (int c = 0; c < D; ++c) {
+      const float4 q4 = *reinterpret_cast<const float4*>(s_qT + c * kDsBlocks + 4 * bgp);
+      const float4 g4 = *reinterpret_cast<const float4*>(s_gT + c * kTile + 4 * kg);
+      const float2 g01 = make_float2(g4.x, g4.y), g23 = make_float2(g4.z, g4.w);
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[u][0] = ffma2(make_float2(qv[u], qv[u]), g01, acc[u][0]);
+        acc[u][1] = ffma2(make_float2(qv[u], qv[u]), g23, acc[u][1]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int blk = i0 + 4 * bgp + u;
+      if (blk < a.Tm)
+        *reinterpret_cast<float4*>(out + (int64_t)blk * a.Np) =
+            make_float4(acc[u][0].x, acc[u][0].y, acc[u][1].x, acc[u][1].y);
+    }
   }
 }
 
@@ -419,7 +490,7 @@ cudaError_t launch_quant_t(const QuantArgs& a, const CUtensorMap& tmVt, cudaStre
   else
     q_quant_kernel<T, D, 128><<<dim3((int)(a.Np / 128), BHq), kThreads, 0, st>>>(a);
   if (a.smooth_q) {
-    const size_t smem = sizeof(float) * D * kTile;
+    const size_t smem = sizeof(float) * D * (kTile + kDsBlocks);
     e = cudaFuncSetAttribute(delta_s_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     delta_s_kernel<T, D><<<dim3(kv_tiles, BHq), kThreads, smem, st>>>(a);

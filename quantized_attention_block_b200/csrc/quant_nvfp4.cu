@@ -6,7 +6,8 @@
 // compensation of SageAttention2), then every group of 16 consecutive elements
 // along the head dimension gets one E4M3 scale, sb = E4M3(amax16 / 6), and E2M1
 // codes E2M1(x / sb).  V is grouped the same way along tokens (the reduction
-// axis of P V).  Every division is an IEEE fp32 division (__fdiv_rn); E2M1 and
+// axis of P V).  Every division is an IEEE fp32 division (__fdiv_rn; per
+// element a reciprocal multiply where it provably gives the same code); E2M1 and
 // E4M3 use round-to-nearest-even with saturation (cvt.rn.satfinite), so codes
 // and scales are bit-exact with the plain definitions.
 //
@@ -32,10 +33,7 @@ __device__ __forceinline__ int sf_byte(int m, int grp) {
 
 // E2M1 codes of x / sd for 8 values (0 when sd == 0), packed low nibble first.
 __device__ __forceinline__ uint32_t encode8_e2m1(const float (&x)[8], float sd) {
-  float y[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) y[e] = sd == 0.0f ? 0.0f : __fdiv_rn(x[e], sd);
-  return cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+  return sd == 0.0f ? 0u : quant_e2m1x8(x, sd, __frcp_rn(sd));
 }
 
 // Encodes row chunk x (8 channels) of a 16-group shared with the partner lane
@@ -207,7 +205,8 @@ __global__ void __launch_bounds__(kThreads) v_quant_nvfp4_kernel(QuantArgs a) {
       lo[u] = x[u];
       hi[u] = x[8 + u];
     }
-    const uint2 codes = make_uint2(encode8_e2m1(lo, sd), encode8_e2m1(hi, sd));
+    const float rd = sd == 0.0f ? 0.0f : __frcp_rn(sd);
+    const uint2 codes = sd == 0.0f ? make_uint2(0u, 0u) : make_uint2(quant_e2m1x8(lo, sd, rd), quant_e2m1x8(hi, sd, rd));
     *reinterpret_cast<uint2*>(sVt + c * (kTile / 2) + grp * 8) = codes;
     s_sf[sf_byte(c, grp)] = (uint8_t)sc;
   }
@@ -243,7 +242,7 @@ cudaError_t launch_quant_nvfp4_t(const QuantArgs& a, cudaStream_t st) {
   else
     q_quant_nvfp4_kernel<T, 128><<<dim3(tiles, BHq), kThreads, 0, st>>>(s);
   if (a.smooth_q) {
-    const size_t smem = sizeof(float) * kF4D * kTile;
+    const size_t smem = sizeof(float) * kF4D * (kTile + kDsBlocks);
     e = cudaFuncSetAttribute(delta_s_kernel<T, kF4D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     delta_s_kernel<T, kF4D><<<dim3(tiles, BHq), kThreads, smem, st>>>(s);
