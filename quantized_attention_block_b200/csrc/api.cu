@@ -122,6 +122,20 @@ bool map_2d_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [B*H][N][D] bf16/fp16 input as a 3D tensor (box 1 x 128 x D, no swizzle):
+// a tile that runs past N reads zeros.
+bool map_3d_input(CUtensorMap* m, const void* base, uint64_t D, uint64_t N, uint64_t BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {D, N, BH};
+  const cuuint64_t strides[2] = {D * 2, N * D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)D, kTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 sage_status fill_view(const sage_params* p, const Dims& d, void* ws, sage_quant_view* v) {
   const Layout L = make_layout(p, d);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -317,11 +331,14 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
   a.dS = view->dS;
   a.ksum = reinterpret_cast<double*>(base + L.ksum);
   a.vamax = reinterpret_cast<unsigned*>(base + L.vamax);
-  CUtensorMap mVt;
-  if (!map_2d_u8(&mVt, view->v8t, (uint64_t)d.Np, (uint64_t)(d.B * d.Hkv * d.D), kTile, (uint32_t)d.D,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
+  QuantMaps m;
+  if (!map_2d_u8(&m.vt, view->v8t, (uint64_t)d.Np, (uint64_t)(d.B * d.Hkv * d.D), kTile, (uint32_t)d.D,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map_3d_input(&m.q, q, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hq)) ||
+      !map_3d_input(&m.k, k, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)) ||
+      !map_3d_input(&m.v, v, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)))
     return SAGE_ERR_CUDA;
-  return from_cuda(launch_quant(a, mVt, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_quant(a, m, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status sage_attn_fwd_quantized(const sage_quant_view* view, void* o, const sage_params* p, void* stream) {

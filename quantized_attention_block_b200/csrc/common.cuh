@@ -63,8 +63,14 @@ struct AttnArgs {
   int32_t* probe_out;
 };
 
+// TMA maps of the preprocessing: the bf16/fp16 inputs as 3D [B*H][N][D] tensors
+// (box 1 x 128 x D) and the transposed E4M3 V output v8t (box D x 128 bytes).
+struct QuantMaps {
+  CUtensorMap q, k, v, vt;
+};
+
 // launchers (defined in the .cu files)
-cudaError_t launch_quant(const QuantArgs& a, const CUtensorMap& tmVt, int is_fp16, cudaStream_t st);
+cudaError_t launch_quant(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st);
 cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, cudaStream_t st);
 cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, cudaStream_t st);

@@ -17,6 +17,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -181,209 +183,199 @@ __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Pass 2a: K (bk-row INT8 blocks of gamma(K)) and V (per-channel E4M3,
-// transposed to [d, Np]) for one 128-token tile.  grid (Np/128, B*Hkv)
-// V is staged in shared memory, each thread encodes 16-token runs of one
-// channel into a 128-byte-swizzled [d x 128] tile, and one TMA store writes
-// the tile to v8t (the same layout the attention kernel's TMA loads read).
+// Pass 2: one 128-row tile of Q, K or V per CTA.  The tile arrives in shared
+// memory by one TMA load (3D map [B*H][N][D]; rows past N read as zeros), so
+// the registers hold no tile and several CTAs per SM keep HBM busy; the
+// threads then sweep the tile in shared memory (block sums, block max, codes).
 template <typename T, int D>
-struct KvSmem {
-  static constexpr int kPitch = D + 8;                          // padded V row (elements)
-  static constexpr uint32_t oVt = 0;                            // [D][128] bytes, 1024-aligned
-  static constexpr uint32_t oV = D * kTile;                     // [128][kPitch] T
-  static constexpr uint32_t kBytes = oV + kTile * kPitch * sizeof(T) + 1024;
-};
+__device__ __forceinline__ bool load_tile(T* dst, const CUtensorMap* map, uint64_t* bar, int row0, int bh) {
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(bar, kTile * D * (uint32_t)sizeof(T));
+    tma_load_3d(dst, map, bar, 0, row0, bh);
+  }
+  return mbar_wait(bar, 0);
+}
 
-template <typename T, int D, int BK>
-__global__ void __launch_bounds__(kThreads) kv_quant_kernel(const __grid_constant__ CUtensorMap tmVt, QuantArgs a) {
-  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, PPB = BK / RG;  // passes per K block
-  constexpr int NKB = kTile / BK;
-  using SL = KvSmem<T, D>;
-  extern __shared__ uint8_t kv_smem_raw[];
-  uint8_t* kv_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(kv_smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sVt = kv_smem + SL::oVt;
-  T* sV = reinterpret_cast<T*>(kv_smem + SL::oV);
-  __shared__ float s_km[D], s_sv[D], s_red[kThreads / 32];
-  __shared__ float s_bmax[NKB];
-  const int bg = blockIdx.y, tile = blockIdx.x;
+__device__ __forceinline__ uint8_t* align128(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 127) & ~uintptr_t(127));
+}
+
+// 8 consecutive elements of a row in shared memory as floats (exact)
+template <typename T>
+__device__ __forceinline__ void lds8(const T* p, float (&x)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  if constexpr (sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+}
+
+// Q (BQ-row blocks, optional block mean) or K (BQ = bk-row blocks, minus km):
+// INT8 codes of x - shift with scale amax_block / 127.
+//   IS_K = false: shift = qbar of the block when smooth_q (written to a.qbar)
+//   IS_K = true:  shift = km = mean_n K (from the fp64 column sums)
+// grid (Np/128, B*H), 256 threads, dynamic smem: 128 x D elements + 128
+template <typename T, int D, int BQ, bool IS_K>
+__global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constant__ CUtensorMap tmX, QuantArgs a) {
+  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BQ, PPB = BQ / RG;
+  extern __shared__ uint8_t qk_smem_raw[];
+  T* sX = reinterpret_cast<T*>(align128(qk_smem_raw));
+  __shared__ double s_sum[kThreads][8];
+  __shared__ float s_shift[NB][D], s_red[kThreads / 32], s_bmax[NB];
+  __shared__ uint64_t bar;
+  const int bh = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
   const int valid = rows_valid(a.N, r0, kTile);
   const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
-
+  const int Tb = IS_K ? a.Tn : a.Tm;
   if (threadIdx.x < D) {
     const int c = threadIdx.x;
-    const float km = a.smooth_k ? __double2float_rn(__ddiv_rn(a.ksum[(int64_t)bg * D + c], (double)a.N)) : 0.0f;
-    const float sv = __fdiv_rn(__uint_as_float(a.vamax[(int64_t)bg * D + c]), 448.0f);
-    s_km[c] = km;
-    s_sv[c] = sv;
-    if (tile == 0) {
-      a.km[(int64_t)bg * D + c] = km;
-      a.s_v[(int64_t)bg * D + c] = sv;
+    if (IS_K) {
+      const float km = a.smooth_k ? __double2float_rn(__ddiv_rn(a.ksum[(int64_t)bh * D + c], (double)a.N)) : 0.0f;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = km;
+      if (tile == 0) a.km[(int64_t)bh * D + c] = km;
+    } else {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = 0.0f;
     }
   }
-  if (threadIdx.x < NKB) s_bmax[threadIdx.x] = 0.0f;
-
-  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
-  const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)bg * a.N * D;
-
-  // ---- V tile -> shared memory (16-byte vectors; rows past N are zero)
+  if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh)) return;
+  if (!IS_K && a.smooth_q) {
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
-    uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (r < valid) u = __ldg(reinterpret_cast<const uint4*>(V + (r0 + r) * D + ch * 8));
-    *reinterpret_cast<uint4*>(sV + r * SL::kPitch + ch * 8) = u;
+    for (int nb = 0; nb < NB; ++nb) {
+      const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
+      double cs[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+      for (int p = nb * PPB; p < (nb + 1) * PPB; ++p) {
+        float x[8];
+        lds8(sX + (rg + p * RG) * D + ch * 8, x);  // rows past N are zero
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cs[e] += (double)x[e];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
+      __syncthreads();
+      if (threadIdx.x < D) {
+        const int c = threadIdx.x;
+        double s = 0.0;
+        for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
+        const float mu = vb > 0 ? __double2float_rn(__ddiv_rn(s, (double)vb)) : 0.0f;
+        s_shift[nb][c] = mu;
+        if (vb > 0) a.qbar[((int64_t)bh * a.Tm + tile * NB + nb) * D + c] = mu;
+      }
+    }
   }
   __syncthreads();
-
-  // ---- K: gamma(K) = K - km, per-block amax, INT8 codes
-  float x[NP][8];
-  float bm[NKB];
+  // block max of |x - shift| over the valid rows
+  float bm[NB];
 #pragma unroll
-  for (int kb = 0; kb < NKB; ++kb) bm[kb] = 0.0f;
+  for (int nb = 0; nb < NB; ++nb) bm[nb] = 0.0f;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int r = rg + p * RG;
     if (r < valid) {
-      load8<T>(K + (r0 + r) * D + ch * 8, x[p]);
+      float x[8];
+      lds8(sX + r * D + ch * 8, x);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        x[p][e] = __fsub_rn(x[p][e], s_km[ch * 8 + e]);
-        bm[p / PPB] = fmaxf(bm[p / PPB], fabsf(x[p][e]));
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[p][e] = 0.0f;
+      for (int e = 0; e < 8; ++e) bm[p / PPB] = fmaxf(bm[p / PPB], fabsf(__fsub_rn(x[e], s_shift[p / PPB][ch * 8 + e])));
     }
   }
 #pragma unroll
-  for (int kb = 0; kb < NKB; ++kb) {
-    const float m = block_max_nonneg(bm[kb], s_red);
-    if (threadIdx.x == 0) s_bmax[kb] = m;
+  for (int nb = 0; nb < NB; ++nb) {
+    const float m = block_max_nonneg(bm[nb], s_red);
+    if (threadIdx.x == 0) s_bmax[nb] = m;
   }
   __syncthreads();
-  float sk[NKB], rk[NKB];
+  float sc[NB], rc[NB];
 #pragma unroll
-  for (int kb = 0; kb < NKB; ++kb) {
-    sk[kb] = __fdiv_rn(s_bmax[kb], 127.0f);
-    rk[kb] = sk[kb] == 0.0f ? 0.0f : __frcp_rn(sk[kb]);
-    const int gb = tile * NKB + kb;
-    if (threadIdx.x == 0 && gb < a.Tn) a.s_k[(int64_t)bg * a.Tn + gb] = sk[kb];
+  for (int nb = 0; nb < NB; ++nb) {
+    sc[nb] = __fdiv_rn(s_bmax[nb], 127.0f);
+    rc[nb] = sc[nb] == 0.0f ? 0.0f : __frcp_rn(sc[nb]);
+    const int gb = tile * NB + nb;
+    if (threadIdx.x == 0 && gb < Tb) (IS_K ? a.s_k : a.s_q)[(int64_t)bh * Tb + gb] = sc[nb];
   }
-  int8_t* k8 = a.k8 + (int64_t)bg * a.Np * D;
+  int8_t* out = (IS_K ? a.k8 : a.q8) + ((int64_t)bh * a.Np + r0) * D;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int r = rg + p * RG;
     int8_t c8[8];
+    if (r < valid) {
+      float x[8];
+      lds8(sX + r * D + ch * 8, x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], sk[p / PPB], rk[p / PPB]) : (int8_t)0;
-    *reinterpret_cast<uint2*>(k8 + (r0 + r) * D + ch * 8) = pack8_i8(c8);
-  }
-
-  // ---- V: E4M3(V / s_v[c]) for 16-token runs of channel c, swizzled [D][128] tile
-  {
-    constexpr int TG = kThreads / D;           // token groups
-    constexpr int RUNS = kTile / 16 / TG;      // 16-token runs per thread
-    const int c = threadIdx.x % D, tg = threadIdx.x / D;
-    const float sv = s_sv[c];
-    const float rv = sv == 0.0f ? 0.0f : __frcp_rn(sv);
+      for (int e = 0; e < 8; ++e) c8[e] = quant_i8(__fsub_rn(x[e], s_shift[p / PPB][ch * 8 + e]), sc[p / PPB], rc[p / PPB]);
+    } else {
 #pragma unroll
-    for (int q = 0; q < RUNS; ++q) {
-      const int run = tg * RUNS + q;
-      uint32_t w[4];
-#pragma unroll
-      for (int u = 0; u < 16; u += 4) {
-        float f[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) f[e] = to_float(sV[(run * 16 + u + e) * SL::kPitch + c]);
-        w[u / 4] = sv == 0.0f ? 0u : quant_e4m3x2(f[0], f[1], sv, rv) | (quant_e4m3x2(f[2], f[3], sv, rv) << 16);
-      }
-      *reinterpret_cast<uint4*>(sVt + c * kTile + ((run ^ (c & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int e = 0; e < 8; ++e) c8[e] = 0;
     }
+    *reinterpret_cast<uint2*>(out + r * D + ch * 8) = pack8_i8(c8);
+  }
+}
+
+// V: E4M3(V / s_v[c]) per channel, transposed to [D][Np].  Each thread encodes
+// 16-token runs of one channel into a 128-byte-swizzled [D x 128] tile; one TMA
+// store writes it to v8t (the layout the attention kernel's TMA loads read).
+// grid (Np/128, B*Hkv), 256 threads, dynamic smem: D x 128 bytes + 128 x D elements
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+    v_quant_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmVt, QuantArgs a) {
+  extern __shared__ uint8_t v_smem_raw[];
+  uint8_t* sVt = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(v_smem_raw) + 1023) & ~uintptr_t(1023));
+  T* sV = reinterpret_cast<T*>(sVt + D * kTile);
+  __shared__ float s_sv[D];
+  __shared__ uint64_t bar;
+  const int bg = blockIdx.y, tile = blockIdx.x;
+  const int64_t r0 = (int64_t)tile * kTile;
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    const float sv = __fdiv_rn(__uint_as_float(a.vamax[(int64_t)bg * D + c]), 448.0f);
+    s_sv[c] = sv;
+    if (tile == 0) a.s_v[(int64_t)bg * D + c] = sv;
+  }
+  if (!load_tile<T, D>(sV, &tmX, &bar, (int)r0, bg)) return;
+  constexpr int TG = kThreads / D;       // token groups
+  constexpr int RUNS = kTile / 16 / TG;  // 16-token runs per thread
+  const int c = threadIdx.x % D, tg = threadIdx.x / D;
+  const float sv = s_sv[c];
+  const float rv = sv == 0.0f ? 0.0f : __frcp_rn(sv);
+#pragma unroll
+  for (int q = 0; q < RUNS; ++q) {
+    const int run = tg * RUNS + q;
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 16; u += 4) {
+      float f[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f[e] = to_float(sV[(run * 16 + u + e) * D + c]);  // rows past N are zero
+      w[u / 4] = sv == 0.0f ? 0u : quant_e4m3x2(f[0], f[1], sv, rv) | (quant_e4m3x2(f[2], f[3], sv, rv) << 16);
+    }
+    *reinterpret_cast<uint4*>(sVt + c * kTile + ((run ^ (c & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   fence_proxy_async_smem();
   __syncthreads();
   if (threadIdx.x == 0) {
     tma_store_2d(&tmVt, sVt, (int)r0, bg * D);
     tma_store_commit_and_wait_read();
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Pass 2b: Q blocks of BQ rows: optional block mean (smooth Q), amax, INT8.
-// grid (Np/BQ, B*Hq)
-template <typename T, int D, int BQ>
-__global__ void __launch_bounds__(kThreads) q_quant_kernel(QuantArgs a) {
-  constexpr int CH = D / 8, RG = kThreads / CH, NP = BQ / RG;
-  __shared__ double s_sum[kThreads][8];
-  __shared__ float s_mean[D], s_red[kThreads / 32];
-  const int bh = blockIdx.y, blk = blockIdx.x;
-  const int64_t r0 = (int64_t)blk * BQ;
-  const int valid = rows_valid(a.N, r0, BQ);
-  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
-  int8_t* q8 = a.q8 + (int64_t)bh * a.Np * D;
-
-  if (valid == 0) {  // padding rows between N and Np
-#pragma unroll
-    for (int p = 0; p < NP; ++p)
-      *reinterpret_cast<uint2*>(q8 + (r0 + rg + p * RG) * D + ch * 8) = make_uint2(0u, 0u);
-    return;
-  }
-  const T* Q = reinterpret_cast<const T*>(a.q) + (int64_t)bh * a.N * D;
-  float x[NP][8];
-#pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
-    if (r < valid) {
-      load8<T>(Q + (r0 + r) * D + ch * 8, x[p]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[p][e] = 0.0f;
-    }
-  }
-  if (a.smooth_q) {
-    double cs[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) cs[e] = 0.0;
-#pragma unroll
-    for (int p = 0; p < NP; ++p)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) cs[e] += (double)x[p][e];  // invalid rows hold 0
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
-    __syncthreads();
-    if (threadIdx.x < D) {
-      const int c = threadIdx.x;
-      double s = 0.0;
-      for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
-      const float mu = __double2float_rn(__ddiv_rn(s, (double)valid));
-      s_mean[c] = mu;
-      a.qbar[((int64_t)bh * a.Tm + blk) * D + c] = mu;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int p = 0; p < NP; ++p)
-      if (rg + p * RG < valid)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[p][e] = __fsub_rn(x[p][e], s_mean[ch * 8 + e]);
-  }
-  float am = 0.0f;
-#pragma unroll
-  for (int p = 0; p < NP; ++p)
-    if (rg + p * RG < valid)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x[p][e]));
-  const float amax = block_max_nonneg(am, s_red);
-  const float s = __fdiv_rn(amax, 127.0f);
-  const float rq = s == 0.0f ? 0.0f : __frcp_rn(s);
-  if (threadIdx.x == 0) a.s_q[(int64_t)bh * a.Tm + blk] = s;
-#pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
-    int8_t c8[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) c8[e] = (r < valid) ? quant_i8(x[p][e], s, rq) : (int8_t)0;
-    *reinterpret_cast<uint2*>(q8 + (r0 + r) * D + ch * 8) = pack8_i8(c8);
   }
 }
 
@@ -467,10 +459,10 @@ __global__ void __launch_bounds__(kThreads) delta_s_kernel(QuantArgs a) {
 }
 
 template <typename T, int D>
-cudaError_t launch_quant_t(const QuantArgs& a, const CUtensorMap& tmVt, cudaStream_t st) {
+cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t st) {
   cudaError_t e;
   const int BHkv = a.B * a.Hkv, BHq = a.B * a.Hq;
-  const int kv_tiles = (int)(a.Np / kTile);
+  const int tiles = (int)(a.Np / kTile);
   if (a.smooth_k) {
     e = cudaMemsetAsync(a.ksum, 0, sizeof(double) * (size_t)BHkv * D, st);
     if (e != cudaSuccess) return e;
@@ -478,33 +470,39 @@ cudaError_t launch_quant_t(const QuantArgs& a, const CUtensorMap& tmVt, cudaStre
   e = cudaMemsetAsync(a.vamax, 0, sizeof(unsigned) * (size_t)BHkv * D, st);
   if (e != cudaSuccess) return e;
   kv_stats_kernel<T, D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(a);
+  const int smem_qk = kTile * D * (int)sizeof(T) + 128;
   {
-    const int smem = (int)KvSmem<T, D>::kBytes;
-    auto kq = a.bk == 64 ? kv_quant_kernel<T, D, 64> : kv_quant_kernel<T, D, 128>;
-    e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kq = a.bk == 64 ? qk_quant_kernel<T, D, 64, true> : qk_quant_kernel<T, D, 128, true>;
+    e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_qk);
     if (e != cudaSuccess) return e;
-    kq<<<dim3(kv_tiles, BHkv), kThreads, smem, st>>>(tmVt, a);
+    kq<<<dim3(tiles, BHkv), kThreads, smem_qk, st>>>(m.k, a);
   }
-  if (a.bq == 64)
-    q_quant_kernel<T, D, 64><<<dim3((int)(a.Np / 64), BHq), kThreads, 0, st>>>(a);
-  else
-    q_quant_kernel<T, D, 128><<<dim3((int)(a.Np / 128), BHq), kThreads, 0, st>>>(a);
+  {
+    const int smem = D * kTile + kTile * D * (int)sizeof(T) + 1024;
+    e = cudaFuncSetAttribute(v_quant_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    v_quant_kernel<T, D><<<dim3(tiles, BHkv), kThreads, smem, st>>>(m.v, m.vt, a);
+  }
+  {
+    auto qq = a.bq == 64 ? qk_quant_kernel<T, D, 64, false> : qk_quant_kernel<T, D, 128, false>;
+    e = cudaFuncSetAttribute(qq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_qk);
+    if (e != cudaSuccess) return e;
+    qq<<<dim3(tiles, BHq), kThreads, smem_qk, st>>>(m.q, a);
+  }
   if (a.smooth_q) {
     const size_t smem = sizeof(float) * D * (kTile + kDsBlocks);
     e = cudaFuncSetAttribute(delta_s_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    delta_s_kernel<T, D><<<dim3(kv_tiles, BHq), kThreads, smem, st>>>(a);
+    delta_s_kernel<T, D><<<dim3(tiles, BHq), kThreads, smem, st>>>(a);
   }
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_quant(const QuantArgs& a, const CUtensorMap& tmVt, int is_fp16, cudaStream_t st) {
-  if (is_fp16)
-    return a.D == 128 ? launch_quant_t<__half, 128>(a, tmVt, st) : launch_quant_t<__half, 64>(a, tmVt, st);
-  return a.D == 128 ? launch_quant_t<__nv_bfloat16, 128>(a, tmVt, st)
-                    : launch_quant_t<__nv_bfloat16, 64>(a, tmVt, st);
+cudaError_t launch_quant(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st) {
+  if (is_fp16) return a.D == 128 ? launch_quant_t<__half, 128>(a, m, st) : launch_quant_t<__half, 64>(a, m, st);
+  return a.D == 128 ? launch_quant_t<__nv_bfloat16, 128>(a, m, st) : launch_quant_t<__nv_bfloat16, 64>(a, m, st);
 }
 
 }  // namespace sage
