@@ -12,7 +12,7 @@
 // not matter), divided in fp64 and rounded once to fp32; every division of
 // the quantisers is an IEEE fp32 division (__fdiv_rn) -- per element it is
 // replaced by a multiplication with the reciprocal wherever that provably
-// gives the same code (quant_i8 / quant_e4m3x2 below) -- and the INT8 rounding
+// gives the same code (quant8_i8 / quant_e4m3x2 below) -- and the INT8 rounding
 // is round-half-to-even.  Do not build with fast-math.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -74,17 +74,28 @@ __device__ __forceinline__ int rows_valid(int N, int64_t r0, int rows) {
 // only arise for codes that are 0 either way.
 constexpr float kBracketLo = 1.0f - 0x1p-21f, kBracketHi = 1.0f + 0x1p-21f;
 
-// rint for |v| < 2^22 in one rounding: the fp32 bits of v + 1.5 * 2^23 (RNE)
-__device__ __forceinline__ int rint_bits(float v) { return __float_as_int(__fadd_rn(v, 12582912.0f)); }
-
-__device__ __forceinline__ int8_t quant_i8(float x, float s, float r) {
-  if (s == 0.0f) return 0;
-  const float y = __fmul_rn(x, r);
-  const int lo = __float_as_int(__fmaf_rn(y, kBracketLo, 12582912.0f));
-  const int hi = __float_as_int(__fmaf_rn(y, kBracketHi, 12582912.0f));
-  int q = (lo == hi) ? lo - 0x4B400000 : __float2int_rn(__fdiv_rn(x, s));
-  q = q > 127 ? 127 : (q < -127 ? -127 : q);
-  return static_cast<int8_t>(q);
+// Eight INT8 codes rint(RN(x[e] / s)) packed little-endian.  |RN(x / s)| <= 127
+// holds by construction (s = RN(amax / 127)), so no clamp is needed, and the code byte is the low byte of the bits of
+// RN(y + 1.5 * 2^23) = 0x4B400000 + rint(y).  s > 0, r = RN(1/s).
+__device__ __forceinline__ uint2 quant8_i8(const float (&x)[8], float s, float r) {
+  uint32_t b[8];
+  bool same = true;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 y = fmul2(make_float2(x[e], x[e + 1]), make_float2(r, r));
+    const float2 lo = ffma2(y, make_float2(kBracketLo, kBracketLo), make_float2(12582912.0f, 12582912.0f));
+    const float2 hi = ffma2(y, make_float2(kBracketHi, kBracketHi), make_float2(12582912.0f, 12582912.0f));
+    b[e] = __float_as_uint(lo.x);
+    b[e + 1] = __float_as_uint(lo.y);
+    same = same && (b[e] == __float_as_uint(hi.x)) && (b[e + 1] == __float_as_uint(hi.y));
+  }
+  if (!same) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) b[e] = (uint32_t)__float2int_rn(__fdiv_rn(x[e], s));
+  }
+  const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+  return make_uint2(w0, w1);
 }
 
 // Two E4M3 codes of x0 / s, x1 / s (lo byte x0); s > 0, r = RN(1/s).
@@ -111,15 +122,6 @@ __device__ __forceinline__ uint32_t quant_e2m1x8(const float (&x)[8], float s, f
 #pragma unroll
   for (int e = 0; e < 8; ++e) q[e] = __fdiv_rn(x[e], s);
   return cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-}
-
-__device__ __forceinline__ uint2 pack8_i8(const int8_t (&c)[8]) {
-  uint2 u;
-  u.x = (uint32_t)(uint8_t)c[0] | ((uint32_t)(uint8_t)c[1] << 8) | ((uint32_t)(uint8_t)c[2] << 16) |
-        ((uint32_t)(uint8_t)c[3] << 24);
-  u.y = (uint32_t)(uint8_t)c[4] | ((uint32_t)(uint8_t)c[5] << 8) | ((uint32_t)(uint8_t)c[6] << 16) |
-        ((uint32_t)(uint8_t)c[7] << 24);
-  return u;
 }
 
 // CTA-wide max of non-negative floats; every thread gets the result.
@@ -231,7 +233,9 @@ __device__ __forceinline__ void lds8(const T* p, float (&x)[8]) {
 //   IS_K = false: shift = qbar of the block when smooth_q (written to a.qbar)
 //   IS_K = true:  shift = km = mean_n K (from the fp64 column sums)
 // grid (Np/128, B*H), 256 threads, dynamic smem: 128 x D elements + 128
-template <typename T, int D, int BQ, bool IS_K>
+//   SHIFT: the shift is applied (smooth_q for Q, smooth_k for K); otherwise it
+//   is identically zero and the block max runs on the raw 16-bit magnitudes.
+template <typename T, int D, int BQ, bool IS_K, bool SHIFT>
 __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constant__ CUtensorMap tmX, QuantArgs a) {
   constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BQ, PPB = BQ / RG;
   extern __shared__ uint8_t qk_smem_raw[];
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
     }
   }
   if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh)) return;
-  if (!IS_K && a.smooth_q) {
+  if (!IS_K && SHIFT) {
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
@@ -288,16 +292,42 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
   __syncthreads();
   // block max of |x - shift| over the valid rows
   float bm[NB];
+  if (SHIFT) {
 #pragma unroll
-  for (int nb = 0; nb < NB; ++nb) bm[nb] = 0.0f;
+    for (int nb = 0; nb < NB; ++nb) bm[nb] = 0.0f;
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
-    if (r < valid) {
-      float x[8];
-      lds8(sX + r * D + ch * 8, x);
+    for (int p = 0; p < NP; ++p) {
+      const int r = rg + p * RG;
+      if (r < valid) {
+        float x[8];
+        lds8(sX + r * D + ch * 8, x);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) bm[p / PPB] = fmaxf(bm[p / PPB], fabsf(__fsub_rn(x[e], s_shift[p / PPB][ch * 8 + e])));
+        for (int e = 0; e < 8; e += 2) {
+          const float2 d = fadd2(make_float2(x[e], x[e + 1]),
+                                 make_float2(-s_shift[p / PPB][ch * 8 + e], -s_shift[p / PPB][ch * 8 + e + 1]));
+          bm[p / PPB] = fmax3(bm[p / PPB], fabsf(d.x), fabsf(d.y));
+        }
+      }
+    }
+  } else {
+    // max |x| on the bit patterns: non-negative bf16 / fp16 values order as
+    // their 16-bit integers (rows past N hold zeros and change nothing)
+    uint32_t mb[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) mb[nb] = 0u;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const uint4 u = *reinterpret_cast<const uint4*>(sX + (rg + p * RG) * D + ch * 8);
+      mb[p / PPB] = __vmaxu2(mb[p / PPB], __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
+                                                   __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu)));
+    }
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const uint32_t m16 = max(mb[nb] & 0xFFFFu, mb[nb] >> 16);
+      if constexpr (std::is_same<T, __nv_bfloat16>::value)
+        bm[nb] = __uint_as_float(m16 << 16);
+      else
+        bm[nb] = __half2float(__ushort_as_half((unsigned short)m16));
     }
   }
 #pragma unroll
@@ -318,17 +348,22 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int r = rg + p * RG;
-    int8_t c8[8];
-    if (r < valid) {
+    uint2 codes = make_uint2(0u, 0u);
+    if (r < valid && sc[p / PPB] != 0.0f) {
       float x[8];
       lds8(sX + r * D + ch * 8, x);
+      if (SHIFT) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) c8[e] = quant_i8(__fsub_rn(x[e], s_shift[p / PPB][ch * 8 + e]), sc[p / PPB], rc[p / PPB]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) c8[e] = 0;
+        for (int e = 0; e < 8; e += 2) {
+          const float2 d = fadd2(make_float2(x[e], x[e + 1]),
+                                 make_float2(-s_shift[p / PPB][ch * 8 + e], -s_shift[p / PPB][ch * 8 + e + 1]));
+          x[e] = d.x;
+          x[e + 1] = d.y;
+        }
+      }
+      codes = quant8_i8(x, sc[p / PPB], rc[p / PPB]);
     }
-    *reinterpret_cast<uint2*>(out + r * D + ch * 8) = pack8_i8(c8);
+    *reinterpret_cast<uint2*>(out + r * D + ch * 8) = codes;
   }
 }
 
@@ -472,7 +507,8 @@ cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t 
   kv_stats_kernel<T, D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(a);
   const int smem_qk = kTile * D * (int)sizeof(T) + 128;
   {
-    auto kq = a.bk == 64 ? qk_quant_kernel<T, D, 64, true> : qk_quant_kernel<T, D, 128, true>;
+    auto kq = a.bk == 64 ? (a.smooth_k ? qk_quant_kernel<T, D, 64, true, true> : qk_quant_kernel<T, D, 64, true, false>)
+                         : (a.smooth_k ? qk_quant_kernel<T, D, 128, true, true> : qk_quant_kernel<T, D, 128, true, false>);
     e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_qk);
     if (e != cudaSuccess) return e;
     kq<<<dim3(tiles, BHkv), kThreads, smem_qk, st>>>(m.k, a);
@@ -484,7 +520,8 @@ cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t 
     v_quant_kernel<T, D><<<dim3(tiles, BHkv), kThreads, smem, st>>>(m.v, m.vt, a);
   }
   {
-    auto qq = a.bq == 64 ? qk_quant_kernel<T, D, 64, false> : qk_quant_kernel<T, D, 128, false>;
+    auto qq = a.bq == 64 ? (a.smooth_q ? qk_quant_kernel<T, D, 64, false, true> : qk_quant_kernel<T, D, 64, false, false>)
+                         : (a.smooth_q ? qk_quant_kernel<T, D, 128, false, true> : qk_quant_kernel<T, D, 128, false, false>);
     e = cudaFuncSetAttribute(qq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_qk);
     if (e != cudaSuccess) return e;
     qq<<<dim3(tiles, BHq), kThreads, smem_qk, st>>>(m.q, a);
