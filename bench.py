@@ -37,6 +37,23 @@ INT8_FP8_PER_BF16 = 2.0  # nominal dense ratio 4.5 / 2.25 PFLOP/s
 FP4_PER_BF16 = 4.0  # nominal dense ratio 9 / 2.25 PFLOP/s
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch of the prefill workload: one ncu capture of attn_i8f8_kernel at B=3
+# (482.3 MB), scaled to B=4 by the number of heads.  Valid only for the kernel
+# source it was taken on (hash below); any other source reports null.
+ATTN_TRAFFIC = {"bytes": 482.3e6 * 4 / 3, "src_sha256_16": "31237b94d47abe89", "workload": "llm_prefill_causal_B4_H32_N4096_d128"}
+
+
+def _attn_traffic(w: W.Workload):
+    import hashlib
+    src = os.path.join(_ROOT, "quantized_attention_block_b200", "csrc", "attn_i8f8.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if sha != ATTN_TRAFFIC["src_sha256_16"] or w.name != ATTN_TRAFFIC["workload"]:
+        return None
+    return ATTN_TRAFFIC["bytes"]
+
+
 def _peaks():
     path = os.path.join(_ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -257,20 +274,21 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
     return res
 
 
-def oracle_sample(w: W.Workload, heads: int, tiles: int, threads: int):
-    """Time the CPU oracle on a bounded sample: quantise `heads` (b, h) pairs
-    and run the attention of the last `tiles` Q tiles of each (the longest rows
-    when causal).  Returns (seconds, attention ops of the sample, description)."""
+def oracle_sample(w: W.Workload, heads: int, tiles: int, threads: int, batches: int = 1):
+    """Time the CPU oracle on a bounded sample: quantise `batches` x `heads`
+    (b, h) pairs and run the attention of the last `tiles` Q tiles of each (the
+    longest rows when causal).  Returns (seconds, attention ops, description)."""
     import numpy as np
 
     import oracle
     from concurrent.futures import ThreadPoolExecutor
 
     G = w.Hq // w.Hkv
-    sw = w.with_(B=1, Hq=heads * G if w.Hq != w.Hkv else heads, Hkv=heads if w.Hq != w.Hkv else heads)
+    sw = w.with_(B=batches, Hq=heads * G if w.Hq != w.Hkv else heads, Hkv=heads if w.Hq != w.Hkv else heads)
     q, k, v = W.make_qkv(sw)
     n_t = -(-w.N // 128)
-    jobs = [(0, h, t * 128, min((t + 1) * 128, w.N)) for h in range(sw.Hq) for t in range(n_t - tiles, n_t)]
+    jobs = [(b, h, t * 128, min((t + 1) * 128, w.N)) for b in range(batches) for h in range(sw.Hq)
+            for t in range(n_t - tiles, n_t)]
     ops = 0.0
     for _, _, r0, r1 in jobs:
         for r in range(r0, r1):
@@ -283,7 +301,7 @@ def oracle_sample(w: W.Workload, heads: int, tiles: int, threads: int):
         list(ex.map(lambda j: oracle.attention_sage_head(quant, j[0], j[1], j[2], j[3], bq=w.bq, bk=w.bk,
                                                         causal=w.causal, sm_scale=w.sm_scale), jobs))
     secs = time.perf_counter() - t_start
-    desc = (f"{sw.Hq} heads of {w.name} (B=1, N={w.N}): full oracle quantisation of those heads + "
+    desc = (f"{batches} x {sw.Hq} heads of {w.name} (N={w.N}): full oracle quantisation of those heads + "
             f"attention of the last {tiles} Q tiles of each ({len(jobs)} tiles), {threads} threads")
     return secs, ops, desc
 
@@ -381,7 +399,7 @@ def main():
                      "peak": peak_tops, "unit": "TFLOP/s", "frac": attn_tops / peak_tops,
                      "peak_source": f"{peak_kind}: bf16 sustained {peaks['bf16_tflops_sustained']} x "
                                     f"{INT8_FP8_PER_BF16} (nominal int8/fp8 : bf16)",
-                     "traffic": None},
+                     "traffic": _attn_traffic(w), "traffic_unit": "bytes per launch"},
         "clocks": res["clocks"], "gpu_launches": res["gpu_launches"], "workloads": extra,
     }
     if "e2e" in res:
@@ -390,9 +408,9 @@ def main():
                        "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
                        "ms_step": e["ms_step"]}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        # about 10-15 s of CPU work on a 16-core host (all heads of batch 0,
-        # the 32 longest Q tiles of each)
-        secs, ops_s, desc = oracle_sample(w, min(32, w.Hkv), 32, threads)
+        # about 10-15 s on a 16-core host: three batches' worth of heads, the 32
+        # longest Q tiles of each
+        secs, ops_s, desc = oracle_sample(w, min(32, w.Hkv), 32, threads, batches=min(3, w.B))
         line["cpu_baseline"] = {"value": ops_s / secs / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
                                 "sample": desc, "seconds": secs}
     if rank == 0:
