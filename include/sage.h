@@ -268,6 +268,14 @@ SAGE_API sage_status sage_debug_qk_nvfp4(const sage_nvfp4_view *view, const sage
                                          int32_t h, int32_t qtile, int32_t ktile, float *out_128x128,
                                          void *stream);
 
+/*
+ * Accuracy probe of the FMA-pipe exponential the attention kernel uses for part
+ * of each row of P (so that not every exp2 waits for the MUFU): y[i] = 2^x[i]
+ * for n device floats, computed by the same device function.  Valid for
+ * -126 <= x <= 100; x < -126 gives 2^-126 or less (the kernel's masked scores).
+ */
+SAGE_API sage_status sage_debug_exp2_poly(const float *x, float *y, int32_t n, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 SAGE_API const char *sage_status_string(sage_status s);
 

@@ -512,6 +512,14 @@ sage_status sage_debug_bounded_wait(uint32_t timeout_us, void* stream) {
   return sage_last_device_error(stream);
 }
 
+sage_status sage_debug_exp2_poly(const float* x, float* y, int32_t n, void* stream) {
+  if (!x || !y || n < 0) return SAGE_ERR_INVALID_ARG;
+  if (n == 0) return SAGE_OK;
+  sage_status s = check_arch();
+  if (s != SAGE_OK) return s;
+  return from_cuda(launch_exp2_poly_probe(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 sage_status sage_debug_f8_accum_probe(float* out8, void* stream) {
   if (!out8 || !aligned16(out8)) return SAGE_ERR_INVALID_ARG;
   sage_status s = check_arch();

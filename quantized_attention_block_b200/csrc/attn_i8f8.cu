@@ -51,6 +51,14 @@ namespace {
 constexpr int kStages = 3;
 constexpr int kThreadsAttn = 512;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
+// Of the 8 element pairs in each 16-key group of the exp loop, those whose bit
+// is set here compute 2^u with exp2_poly2 (FMA/ALU pipes) instead of ex2 (MUFU).
+// Measured on B200: every split tried (1/4, 3/8, 1/2 of the pairs) was slower
+// than MUFU only -- the loop is bound by issue slots, not by the MUFU rate.
+#ifndef SAGE_POLY_PAIRS
+#define SAGE_POLY_PAIRS 0x00
+#endif
+constexpr unsigned kPolyPairs = SAGE_POLY_PAIRS;
 
 // per-warpgroup register budgets after setmaxnreg (sum x 128 <= 65536)
 constexpr uint32_t kRegsProducer = 40, kRegsSoftmax = 192, kRegsCorrection = 88;
@@ -451,8 +459,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             u0 = ffma2(fadd2(y0, neg_magic), make_float2(sc, sc), make_float2(-mm, -mm));
             u1 = ffma2(fadd2(y1, neg_magic), make_float2(sc, sc), make_float2(-mm, -mm));
           }
-          const float2 p0 = make_float2(ex2_approx(u0.x), ex2_approx(u0.y));
-          const float2 p1 = make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
+          // pairs selected by kPolyPairs take the FMA-pipe exponential, the rest MUFU
+          const float2 p0 = ((kPolyPairs >> (e / 2)) & 1) ? exp2_poly2(u0)
+                                                          : make_float2(ex2_approx(u0.x), ex2_approx(u0.y));
+          const float2 p1 = ((kPolyPairs >> (e / 2 + 1)) & 1) ? exp2_poly2(u1)
+                                                              : make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
           rs[e / 2] = fadd2(rs[e / 2], p0);
           rs[e / 2 + 1] = fadd2(rs[e / 2 + 1], p1);
           w[e / 4] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
@@ -772,6 +783,18 @@ __global__ void __launch_bounds__(128, 1) f8_accum_probe_kernel(float* out) {
   }
 }
 
+// exp2_poly2 on an array (accuracy test of the FMA-pipe exponential).
+__global__ void exp2_poly_probe_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], x[i])).x;
+  }
+}
+
 // A wait nobody ends: the bounded wait gives up, records the timeout, returns.
 __global__ void bounded_wait_probe_kernel() {
   __shared__ uint64_t bar;
@@ -843,6 +866,12 @@ cudaError_t launch_f8_accum_probe(float* out, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(f8_accum_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   f8_accum_probe_kernel<<<1, 128, smem, st>>>(out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_exp2_poly_probe(const float* x, float* y, int n, cudaStream_t st) {
+  const int pairs = (n + 1) / 2;
+  exp2_poly_probe_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y, n);
   return cudaGetLastError();
 }
 

@@ -75,6 +75,7 @@ cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CU
                              const CUtensorMap& tmV, cudaStream_t st);
 cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(cudaStream_t st);
+cudaError_t launch_exp2_poly_probe(const float* x, float* y, int n, cudaStream_t st);
 cudaError_t launch_f8_accum_probe(float* out, cudaStream_t st);
 cudaError_t launch_quant_nvfp4(const QuantArgs& a, int is_fp16, cudaStream_t st);
 cudaError_t launch_attn_nvfp4(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,

@@ -27,7 +27,7 @@ EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized",
             "sage_debug_qk_int32", "sage_last_device_error", "sage_debug_bounded_wait",
             "sage_status_string", "sage_attn_fwd_noalloc", "sage_debug_f8_accum_probe",
             "sage_nvfp4_workspace_bytes", "sage_quant_nvfp4", "sage_attn_fwd_nvfp4_quantized",
-            "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4")
+            "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4", "sage_debug_exp2_poly")
 
 
 class SageError(RuntimeError):
@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
         L.sage_attn_fwd_nvfp4_quantized.argtypes = [F, vp, P, vp]
         L.sage_attn_fwd_nvfp4.argtypes = [vp, vp, vp, vp, P, vp, ctypes.c_size_t, vp]
         L.sage_debug_qk_nvfp4.argtypes = [F, P, i32, i32, i32, i32, vp, vp]
+        L.sage_debug_exp2_poly.argtypes, L.sage_debug_exp2_poly.restype = [vp, vp, i32, vp], ctypes.c_int
         for n in ("sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd", "sage_debug_qk_int32",
                   "sage_last_device_error", "sage_debug_bounded_wait", "sage_quant_nvfp4",
                   "sage_attn_fwd_nvfp4_quantized", "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4"):
@@ -261,6 +262,13 @@ def sage_debug_qk_nvfp4(view: SageNvfp4View, p: SageParams, b: int, h: int, qtil
     _check(lib().sage_debug_qk_nvfp4(ctypes.byref(view), ctypes.byref(p), b, h, qtile, ktile, _ptr(out),
                                      _stream(stream)), "sage_debug_qk_nvfp4")
     return out
+
+
+def sage_debug_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x of a float32 device tensor through the kernel's FMA-pipe exponential."""
+    y = torch.empty_like(x)
+    _check(lib().sage_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "sage_debug_exp2_poly")
+    return y
 
 
 def nvfp4_view_tensors(view: SageNvfp4View, p: SageParams, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:

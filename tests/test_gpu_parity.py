@@ -169,3 +169,16 @@ def test_fp8_accumulator_precision_probe():
     assert got[2] == exact[2] and got[3] == 256.0 and got[4] == 32.0, got
     bits = [int(-np.log2(abs(g - round(g)) or 2.0 ** -40)) if g != round(g) else None for g in got]
     print("f8 accumulator probe:", got.tolist(), "exact:", [float(x) == float(y) for x, y in zip(got, exact)], bits)
+
+
+def test_fma_pipe_exp2_accuracy():
+    """The polynomial exp2 the softmax uses for part of each row: relative error
+    against fp64 exp2 below 1.2e-5 over the range the kernel feeds it (scores
+    minus the row max plus log2 448), exact zero-ish for masked scores."""
+    x = torch.cat([torch.linspace(-125.0, 9.0, 2_000_001), torch.tensor([0.0, 1.0, -1.0, 8.807354922057604])])
+    y = sage.sage_debug_exp2_poly(x.cuda()).cpu().double()
+    ref = torch.exp2(x.double())
+    rel = ((y - ref).abs() / ref).max().item()
+    assert rel < 1.2e-5, rel
+    masked = sage.sage_debug_exp2_poly(torch.tensor([-float("inf"), -1e30, -500.0]).cuda()).cpu()
+    assert torch.all(masked >= 0) and torch.all(masked <= 2.0 ** -125)
