@@ -51,6 +51,11 @@ namespace {
 constexpr int kStages = 3;
 constexpr int kThreadsAttn = 512;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
+// S starts from the magic fill and gets it back after every read.  (Measured:
+// this beats fresh int32 accumulators converted in the softmax by 10-16%.  The
+// exp argument keeps the exact (y - 12582912) a - m: folding the offset into
+// one FMA, y a - (12582912 a + m), rounds y a at 2^23 magnitude and broke the
+// 1e-2 output tolerance on the prefill recipe.)
 // Of the 8 element pairs in each 16-key group of the exp loop, those whose bit
 // is set here compute 2^u with exp2_poly2 (FMA/ALU pipes) instead of ex2 (MUFU).
 // Measured on B200: every split tried (1/4, 3/8, 1/2 of the pairs) was slower
@@ -400,6 +405,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const int col = col0 + c;
+          // -inf as y (or, raw int32 without the fill, the value whose y is -inf)
           if (col >= a.N || (CAUSAL && col > qrow)) s[c] = __float_as_uint(-INFINITY);
         }
       }
@@ -466,7 +472,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                                               : make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
           rs[e / 2] = fadd2(rs[e / 2], p0);
           rs[e / 2 + 1] = fadd2(rs[e / 2 + 1], p1);
-          w[e / 4] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
+          w[e / 4] = cvt_e4m3x4(p0.x, p0.y, p1.x, p1.y);
         }
         *reinterpret_cast<uint4*>(myP + ((grp ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }

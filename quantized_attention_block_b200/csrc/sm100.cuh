@@ -392,6 +392,18 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float f0, float f1, float f2, flo
   return r;
 }
 
+// Four floats -> four E4M3 codes in one word (f0 in bits 0-7 ... f3 in 24-31).
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float f0, float f1, float f2, float f3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(f0), "f"(f1), "f"(f2), "f"(f3));
+  return r;
+}
+
 // One float -> E4M3 code (round-to-nearest-even, saturate to +-448).
 __device__ __forceinline__ uint32_t cvt_e4m3(float x) { return cvt_e4m3x2(x, 0.0f) & 0xFFu; }
 
