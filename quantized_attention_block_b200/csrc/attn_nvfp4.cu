@@ -68,14 +68,14 @@ struct SmemF4 {
   static constexpr uint32_t oK = oQ + 2 * kT;
   static constexpr uint32_t oV = oK + kStF4 * kT;
   static constexpr uint32_t oP = oV + kStF4 * kT;
-  static constexpr uint32_t oSFQ = oP + 2 * kT;
+  static constexpr uint32_t oSFQ = oP + 4 * kT;  // P: [tile][2 buffers]
   static constexpr uint32_t oSFK = oSFQ + 2 * kSF;
   static constexpr uint32_t oSFV = oSFK + kStF4 * kSF;
   static constexpr uint32_t oSFP = oSFV + kStF4 * kSF;
-  static constexpr uint32_t oR = oSFP + 2 * kSF;   // float[2][128] rescale factor r
-  static constexpr uint32_t oL = oR + 2 * 128 * 4;  // float[2][128] final 1 / (2688 l exp2(m - E))
+  static constexpr uint32_t oR = oSFP + 4 * kSF;   // float[tile][buffer][128] rescale factor r
+  static constexpr uint32_t oL = oR + 4 * 128 * 4;  // float[2][128] final 1 / (2688 l exp2(m - E))
   static constexpr uint32_t oBar = oL + 2 * 128 * 4;
-  static constexpr uint32_t kNumBars = 1 + 3 * kStF4 + 1 + 6 * 2 + 1;
+  static constexpr uint32_t kNumBars = 1 + 3 * kStF4 + 1 + 2 + 4 + 4 + 2 + 2 + 2 + 1;
   static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = oTmem + 16 + 1024;
 };
@@ -87,7 +87,8 @@ struct BarsF4 {
   uint64_t* kv_empty;  // [kStF4]
   uint64_t* s_free;    // S columns read by the softmax that owned them (128 arrivals)
   uint64_t* s_full;    // [2] Q K^T of tile i in S
-  uint64_t* p_full;    // [2] P^_i, its scales and r_i written (128 arrivals)
+  uint64_t* p_full;    // [tile][buffer j & 1] P^_i(j), its scales and r_i(j) written (128 arrivals)
+  uint64_t* p_empty;   // [tile][buffer] the P V that read that buffer retired
   uint64_t* ot_full;   // [2] P V of tile i retired
   uint64_t* o_ready;   // [2] A_i rescaled for the next P V (128 arrivals)
   uint64_t* l_ready;   // [2] final normaliser of tile i in shared memory (128 arrivals)
@@ -138,7 +139,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
   bar.s_free = bar.kv_empty + kStF4;
   bar.s_full = bar.s_free + 1;
   bar.p_full = bar.s_full + 2;
-  bar.ot_full = bar.p_full + 2;
+  bar.p_empty = bar.p_full + 4;
+  bar.ot_full = bar.p_empty + 4;
   bar.o_ready = bar.ot_full + 2;
   bar.l_ready = bar.o_ready + 2;
   bar.mma_done = bar.l_ready + 2;
@@ -173,7 +175,10 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
     mbar_init(bar.s_free, 128);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar.s_full[i], 1);
-      mbar_init(&bar.p_full[i], 128);
+      mbar_init(&bar.p_full[2 * i], 128);
+      mbar_init(&bar.p_full[2 * i + 1], 128);
+      mbar_init(&bar.p_empty[2 * i], 1);
+      mbar_init(&bar.p_empty[2 * i + 1], 1);
       mbar_init(&bar.ot_full[i], 1);
       mbar_init(&bar.o_ready[i], 128);
       mbar_init(&bar.l_ready[i], 128);
@@ -286,7 +291,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
           for (int i = 0; i < 2; ++i) {
             const int jp = next_pv[i];
             const int s = jp % kStF4;
-            if (jp < nTi[i] && issued_qk[i] > jp && mbar_test_wait(smem_u32(&bar.p_full[i]), jp & 1) &&
+            if (jp < nTi[i] && issued_qk[i] > jp &&
+                mbar_test_wait(smem_u32(&bar.p_full[i * 2 + (jp & 1)]), (jp >> 1) & 1) &&
                 mbar_test_wait(smem_u32(&bar.v_full[s]), (jp / kStF4) & 1) &&
                 (jp == 0 || mbar_test_wait(smem_u32(&bar.o_ready[i]), (jp - 1) & 1))) {
               tc_fence_after();
@@ -296,14 +302,15 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
                 sfv_next = jp + 1;
               }
               for (int kk = 0; kk < 2; ++kk)
-                tmem_cp_sf(tmem + col_sfp(i, kk), sf_desc(smem_u32(sSFP + i * L::kSF + kk * 512)));
-              const uint32_t aP = smem_u32(sP + i * L::kT), aV = smem_u32(sV + s * L::kT);
+                tmem_cp_sf(tmem + col_sfp(i, kk), sf_desc(smem_u32(sSFP + (i * 2 + (jp & 1)) * L::kSF + kk * 512)));
+              const uint32_t aP = smem_u32(sP + (i * 2 + (jp & 1)) * L::kT), aV = smem_u32(sV + s * L::kT);
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk)
                 mma_nvf4(tmem + kColA + 128 * i, make_sdesc(aP + kk * 32, 512, kSwizzle64B),
                          make_sdesc(aV + kk * 32, 512, kSwizzle64B), kIdesc, tmem + col_sfp(i, kk),
                          tmem + col_sfv(s, kk), (jp > 0 || kk > 0) ? 1u : 0u);
               mma_commit(&bar.ot_full[i]);
+              mma_commit(&bar.p_empty[i * 2 + (jp & 1)]);
               next_pv[i] = jp + 1;
               progress = true;
             }
@@ -342,8 +349,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
     const uint32_t tS = tmem + kColS + ((uint32_t)(quarter * 32) << 16);
     const int qblk = min((int)(qrow / a.bq), a.Tm - 1);
     const float* dsr = HAS_DS ? a.dS + ((int64_t)bh * a.Tm + qblk) * a.Np : nullptr;
-    uint8_t* myP = sP + ti * L::kT + row * 64;
-    uint32_t* mySF = reinterpret_cast<uint32_t*>(sSFP + ti * L::kSF) + 4 * lane + quarter;
+    uint8_t* myP0 = sP + ti * 2 * L::kT + row * 64;  // buffer b at + b * kT
+    uint32_t* mySF0 = reinterpret_cast<uint32_t*>(sSFP + ti * 2 * L::kSF) + 4 * lane + quarter;
     const float sl2 = a.scale_log2;
     float m = -INFINITY, l = 0.0f, E = 0.0f;
     bool ok = true;
@@ -388,8 +395,10 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
       const float m_new = fmaxf(m, mt);
       const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
       const bool keep = mt >= m_new - kDropLog2;  // false only for a row far below the running max
-      // P^_i and its scales are single-buffered: P V(j-1) must have read them
-      if (j > 0 && !(ok = mbar_wait_warp(&bar.ot_full[ti], (j - 1) & 1))) break;
+      // P buffer (j & 1) and its scales are free once P V(j - 2) retired
+      if (j >= 2 && !(ok = mbar_wait_warp(&bar.p_empty[ti * 2 + (j & 1)], ((j >> 1) - 1) & 1))) break;
+      uint8_t* myP = myP0 + (j & 1) * L::kT;
+      uint32_t* mySF = mySF0 + (j & 1) * (L::kSF / 4);
       const float mm = keep ? mt - kLog2_2688 : INFINITY;  // P2 = exp2(t - mm); dropped rows give 0
       float2 rs[4];
 #pragma unroll
@@ -412,9 +421,11 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
           }
           const float gm = fmax3(fmax3(fmax3(p[0], p[1], p[2]), fmax3(p[3], p[4], p[5]), fmax3(p[6], p[7], p[8])),
                                  fmax3(p[9], p[10], p[11]), fmax3(p[12], p[13], fmaxf(p[14], p[15])));
-          const uint32_t sc = cvt_e4m3(__fdiv_rn(gm, 6.0f));
+          // s_P2 = E4M3(amax16 / 6) and 1 / s_P2 without IEEE division steps (a
+          // code can differ from the divided one only at an exact midpoint)
+          const uint32_t sc = cvt_e4m3(gm * (1.0f / 6.0f));
           const float sd = e4m3_value(sc);
-          const float inv = sd > 0.0f ? __frcp_rn(sd) : 0.0f;
+          const float inv = sd > 0.0f ? rcp_approx(sd) : 0.0f;
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
             const float2 q = fmul2(make_float2(p[e], p[e + 1]), make_float2(inv, inv));
@@ -442,10 +453,10 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
         r = (j == 0) ? 1.0f : ex2_approx(E - mt);
         E = mt;
       }  // a dropped row leaves l as it is (alpha == 1 there; its share is < 2^-25 of l)
-      s_r[ti * 128 + row] = r;
+      s_r[(ti * 2 + (j & 1)) * 128 + row] = r;
       tc_fence_before();
       fence_proxy_async_smem();
-      mbar_arrive(&bar.p_full[ti]);
+      mbar_arrive(&bar.p_full[ti * 2 + (j & 1)]);
       m = m_new;
     }
     // out = A exp2(E - m) / (2688 l)
@@ -463,11 +474,11 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
     for (int j = 0; j < nT && ok; ++j) {
       for (int i = 0; i < 2; ++i) {
         if (j >= nTi[i]) continue;
-        if (!(ok = mbar_wait_warp(&bar.p_full[i], j & 1))) break;
+        if (!(ok = mbar_wait_warp(&bar.p_full[i * 2 + (j & 1)], (j >> 1) & 1))) break;
         if (j == 0) continue;
         if (!(ok = mbar_wait_warp(&bar.ot_full[i], (j - 1) & 1))) break;
         tc_fence_after();
-        const float r = s_r[i * 128 + row];
+        const float r = s_r[(i * 2 + (j & 1)) * 128 + row];
         if (__any_sync(0xffffffffu, r != 1.0f)) {
           const uint32_t tA = tmem + kColA + 128 * i + lane_off;
 #pragma unroll

@@ -368,6 +368,12 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Two floats -> two E4M3 codes (round-to-nearest-even, saturate to +-448);
 // `lo` lands in bits 0-7, `hi` in bits 8-15.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
