@@ -389,16 +389,24 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       }
       const bool need_mask = (col0 + kTile > a.N) || (CAUSAL && j == qtile);
       float mx;
+      // with delta_S: x = (y - 12582912) + delta_S sm_scale log2 e / a in place, so
+      // that the score is t = x a (a >= 1e-30 here keeps the quotient finite; a
+      // zero scale only multiplies zero dot products)
+      const float ad_lo = fmaxf(a_lo, 1e-30f), ad_hi = fmaxf(a_hi, 1e-30f);
       if (HAS_DS) {
-        // t = (y - 12582912) a + delta_S sm_scale log2 e, in place
+        const float k_lo = sl2 / ad_lo, k_hi = sl2 / ad_hi;
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float sc = c < 64 ? a_lo : a_hi;
-          const float2 x = fadd2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), neg_magic);
-          const float2 ds = *reinterpret_cast<const float2*>(dsr + c);
-          const float2 t = ffma2(x, make_float2(sc, sc), fmul2(ds, make_float2(sl2, sl2)));
-          s[c] = __float_as_uint(t.x);
-          s[c + 1] = __float_as_uint(t.y);
+        for (int c = 0; c < 128; c += 4) {
+          const float kc = c < 64 ? k_lo : k_hi;
+          const float4 ds = *reinterpret_cast<const float4*>(dsr + c);
+          const float2 x0 = ffma2(make_float2(ds.x, ds.y), make_float2(kc, kc),
+                                  fadd2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), neg_magic));
+          const float2 x1 = ffma2(make_float2(ds.z, ds.w), make_float2(kc, kc),
+                                  fadd2(make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])), neg_magic));
+          s[c] = __float_as_uint(x0.x);
+          s[c + 1] = __float_as_uint(x0.y);
+          s[c + 2] = __float_as_uint(x1.x);
+          s[c + 3] = __float_as_uint(x1.y);
         }
       }
       if (need_mask) {
@@ -410,16 +418,19 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
       }
       if (HAS_DS) {
-        // row max: 8 independent 3-input chains, then a short tree (max is exact)
+        // row max of t = x a per 64-key half (a > 0 keeps the order of x)
         float mx8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 16)
+        for (int c = 0; c < 64; c += 8)
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
+          for (int k = 0; k < 4; ++k) {
             mx8[k] = fmax3(mx8[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
-        mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+            mx8[4 + k] = fmax3(mx8[4 + k], __uint_as_float(s[64 + c + 2 * k]), __uint_as_float(s[64 + c + 2 * k + 1]));
+          }
+        mx = fmaxf(fmax3(mx8[0], mx8[1], fmaxf(mx8[2], mx8[3])) * ad_lo,
+                   fmax3(mx8[4], mx8[5], fmaxf(mx8[6], mx8[7])) * ad_hi);
       } else {
         // y is monotonic in acc: take the max of each 64-key half on y and scale
         // only the two maxima
@@ -458,8 +469,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           const float2 y0 = make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1]));
           const float2 y1 = make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
           if (HAS_DS) {
-            u0 = fadd2(y0, make_float2(-mm, -mm));
-            u1 = fadd2(y1, make_float2(-mm, -mm));
+            const float sc = c < 64 ? ad_lo : ad_hi;
+            u0 = ffma2(y0, make_float2(sc, sc), make_float2(-mm, -mm));
+            u1 = ffma2(y1, make_float2(sc, sc), make_float2(-mm, -mm));
           } else {
             const float sc = c < 64 ? a_lo : a_hi;
             u0 = ffma2(fadd2(y0, neg_magic), make_float2(sc, sc), make_float2(-mm, -mm));

@@ -72,7 +72,9 @@ struct SmemF4 {
   static constexpr uint32_t oSFK = oSFQ + 2 * kSF;
   static constexpr uint32_t oSFV = oSFK + kStF4 * kSF;
   static constexpr uint32_t oSFP = oSFV + kStF4 * kSF;
-  static constexpr uint32_t oR = oSFP + 4 * kSF;   // float[tile][buffer][128] rescale factor r
+  static constexpr uint32_t kDS = 2 * 2 * 128 * 4;  // delta_S rows of one key tile: [tile][Q block][128]
+  static constexpr uint32_t oDS = oSFP + 4 * kSF;   // kStF4
+  static constexpr uint32_t oR = oDS + kStF4 * kDS;  // float[tile][buffer][128] rescale factor r
   static constexpr uint32_t oL = oR + 4 * 128 * 4;  // float[2][128] final 1 / (2688 l exp2(m - E))
   static constexpr uint32_t oBar = oL + 2 * 128 * 4;
   static constexpr uint32_t kNumBars = 1 + 3 * kStF4 + 1 + 2 + 4 + 4 + 2 + 2 + 2 + 1;
@@ -206,6 +208,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
       const int64_t qhead = (int64_t)bh * a.Np;
       const int krow0 = (int)((int64_t)bg * a.Np);
       const int vrow = bg * 128;
+      const int ds_rows = kTile / a.bq;  // Q blocks per tile (1 or 2)
+      const uint32_t ds_bytes = (uint32_t)((nTi[0] > 0) + (nTi[1] > 0)) * ds_rows * 512;
       mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kT + L::kSF : 0u) + (nTi[1] > 0 ? L::kT + L::kSF : 0u));
       for (int i = 0; i < 2; ++i)
         if (nTi[i] > 0) {
@@ -220,9 +224,19 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
         if (j >= kStF4) ok = mbar_wait(&bar.kv_empty[s], ((j / kStF4) + 1) & 1);
         if (!ok) break;
         const int64_t kvt = (int64_t)bg * tiles_per_head + j;
-        mbar_expect_tx(&bar.k_full[s], L::kT + L::kSF);
+        mbar_expect_tx(&bar.k_full[s], L::kT + L::kSF + (HAS_DS ? ds_bytes : 0u));
         tma_load_2d(sK + s * L::kT, &tmK, &bar.k_full[s], 0, krow0 + j * kTile);
         bulk_load_1d(sSFK + s * L::kSF, a.sfk + kvt * 1024, L::kSF, &bar.k_full[s]);
+        if (HAS_DS) {
+          // delta_S[b, h, Q block, keys of tile j] for the Q blocks of both tiles
+          for (int i = 0; i < 2; ++i)
+            for (int hb = 0; hb < ds_rows; ++hb)
+              if (nTi[i] > 0) {
+                const int blk = min((2 * pr + i) * ds_rows + hb, a.Tm - 1);
+                bulk_load_1d(smem + L::oDS + s * L::kDS + (i * 2 + hb) * 512,
+                             a.dS + ((int64_t)bh * a.Tm + blk) * a.Np + (int64_t)j * kTile, 512, &bar.k_full[s]);
+              }
+        }
         mbar_expect_tx(&bar.v_full[s], L::kT + L::kSF);
         tma_load_2d(sV + s * L::kT, &tmV, &bar.v_full[s], j * (kTile / 2), vrow);
         bulk_load_1d(sSFV + s * L::kSF, a.sfv + kvt * 1024, L::kSF, &bar.v_full[s]);
@@ -347,8 +361,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
     const int qtile = 2 * pr + ti;
     const int64_t qrow = (int64_t)qtile * kTile + row;
     const uint32_t tS = tmem + kColS + ((uint32_t)(quarter * 32) << 16);
-    const int qblk = min((int)(qrow / a.bq), a.Tm - 1);
-    const float* dsr = HAS_DS ? a.dS + ((int64_t)bh * a.Tm + qblk) * a.Np : nullptr;
+    const int ds_half = (a.bq == 64 && row >= 64) ? 1 : 0;  // warp-uniform
+    const float* sDS = reinterpret_cast<const float*>(smem + L::oDS);
     uint8_t* myP0 = sP + ti * 2 * L::kT + row * 64;  // buffer b at + b * kT
     uint32_t* mySF0 = reinterpret_cast<uint32_t*>(sSFP + ti * 2 * L::kSF) + 4 * lane + quarter;
     const float sl2 = a.scale_log2;
@@ -366,14 +380,18 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
       tc_fence_before();
       mbar_arrive(bar.s_free);
       const int col0 = j * kTile;
-      // t = (S + delta_S) * sm_scale * log2 e
+      // x = S + delta_S (the scores are t = x sm_scale log2 e; the scale is
+      // applied to the max and inside the exponent's FMA)
+      if (HAS_DS) {
+        const float* dsr = sDS + (j % kStF4) * (L::kDS / 4) + (ti * 2 + ds_half) * 128;
+        if (!(ok = mbar_wait_warp(&bar.k_full[j % kStF4], (j / kStF4) & 1))) break;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        float2 x = make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-        if (HAS_DS) x = fadd2(x, __ldg(reinterpret_cast<const float2*>(dsr + col0 + c)));
-        x = fmul2(x, make_float2(sl2, sl2));
-        s[c] = __float_as_uint(x.x);
-        s[c + 1] = __float_as_uint(x.y);
+        for (int c = 0; c < 128; c += 2) {
+          const float2 x = fadd2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                 *reinterpret_cast<const float2*>(dsr + c));
+          s[c] = __float_as_uint(x.x);
+          s[c + 1] = __float_as_uint(x.y);
+        }
       }
       const bool need_mask = (col0 + kTile > a.N) || (CAUSAL && j == qtile);
       if (need_mask) {
@@ -391,7 +409,7 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           mx8[k] = fmax3(mx8[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
-      const float mt = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+      const float mt = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])) * sl2;
       const float m_new = fmaxf(m, mt);
       const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
       const bool keep = mt >= m_new - kDropLog2;  // false only for a row far below the running max
@@ -413,8 +431,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
           float p[16];
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
-            const float2 u = fadd2(make_float2(__uint_as_float(s[c0 + e]), __uint_as_float(s[c0 + e + 1])),
-                                   make_float2(-mm, -mm));
+            const float2 u = ffma2(make_float2(__uint_as_float(s[c0 + e]), __uint_as_float(s[c0 + e + 1])),
+                                   make_float2(sl2, sl2), make_float2(-mm, -mm));
             p[e] = ex2_approx(u.x);
             p[e + 1] = ex2_approx(u.y);
             rs[e / 4] = fadd2(rs[e / 4], make_float2(p[e], p[e + 1]));
