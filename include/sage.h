@@ -113,6 +113,11 @@ SAGE_API size_t sage_workspace_bytes(const sage_params *p);
  * q, k, v: device [B,H,N,d] in p->dtype.  Fills *view (host struct) with
  * pointers into `workspace`.  Quantised tensors and scales are bit-exact with
  * the plain definitions above.
+ * For d = 128, K and V are read from HBM once when the ceil(N/128) tiles of
+ * one head fit twice in the CTAs the GPU holds at once (tiles wait in shared
+ * memory for their head's km / s_v); otherwise a statistics pass runs first.
+ * Both give the same bytes.  A wait that runs out (a GPU shared with a stalled kernel)
+ * records SAGE_ERR_TIMEOUT for sage_last_device_error.
  */
 SAGE_API sage_status sage_quant_qkv(const void *q, const void *k, const void *v, const sage_params *p,
                            void *workspace, size_t workspace_bytes,
@@ -275,6 +280,14 @@ SAGE_API sage_status sage_debug_qk_nvfp4(const sage_nvfp4_view *view, const sage
  * -126 <= x <= 100; x < -126 gives 2^-126 or less (the kernel's masked scores).
  */
 SAGE_API sage_status sage_debug_exp2_poly(const float *x, float *y, int32_t n, void *stream);
+
+/*
+ * Test hook: on = 1 makes sage_quant_qkv (and the calls built on it) take the
+ * two-pass K/V path (statistics kernel, then the code kernels) in this
+ * process; on = 0 restores the default choice.  Not thread-safe with
+ * concurrent sage_quant_qkv calls.  SAGE_ERR_INVALID_ARG for other values.
+ */
+SAGE_API sage_status sage_debug_kv_quant_two_pass(int32_t on);
 
 /* Human-readable name of a status code (static storage). */
 SAGE_API const char *sage_status_string(sage_status s);

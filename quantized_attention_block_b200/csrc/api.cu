@@ -27,8 +27,11 @@ struct Dims {
 };
 
 struct Layout {
-  size_t q8, k8, v8t, s_q, s_k, s_v, km, ksum, vamax, qbar, dS, total;
+  size_t q8, k8, v8t, s_q, s_k, s_v, km, ksum, vamax, kv_sync, kv_sync_end, qbar, dS, total;
 };
+
+// 1: sage_quant_qkv always takes the two-pass K/V path (sage_debug_kv_quant_two_pass)
+int g_kv_two_pass = 0;
 
 sage_status check_params(const sage_params* p, Dims* d) {
   if (!p) return SAGE_ERR_INVALID_ARG;
@@ -71,8 +74,11 @@ Layout make_layout(const sage_params* p, const Dims& d) {
   L.s_k = take(4 * (size_t)(d.B * d.Hkv * d.Tn));
   L.s_v = take(4 * (size_t)(d.B * d.Hkv * d.D));
   L.km = take(4 * (size_t)(d.B * d.Hkv * d.D));
+  // ksum, vamax, kv_sync consecutive: the one-read K/V kernel zeroes them with one memset
   L.ksum = take(8 * (size_t)(d.B * d.Hkv * d.D));
   L.vamax = take(4 * (size_t)(d.B * d.Hkv * d.D));
+  L.kv_sync = take(4 * (size_t)(1 + 2 * d.B * d.Hkv));
+  L.kv_sync_end = L.kv_sync + 4 * (size_t)(1 + 2 * d.B * d.Hkv);
   if (p->smooth_q) {
     L.qbar = take(4 * (size_t)(d.B * d.Hq * d.Tm * d.D));
     L.dS = take(4 * (size_t)(d.B * d.Hq * d.Tm * d.Np));
@@ -331,6 +337,8 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
   a.dS = view->dS;
   a.ksum = reinterpret_cast<double*>(base + L.ksum);
   a.vamax = reinterpret_cast<unsigned*>(base + L.vamax);
+  a.kv_sync = g_kv_two_pass ? nullptr : reinterpret_cast<int*>(base + L.kv_sync);
+  a.kv_zero_bytes = L.kv_sync_end - L.ksum;
   QuantMaps m;
   if (!map_2d_u8(&m.vt, view->v8t, (uint64_t)d.Np, (uint64_t)(d.B * d.Hkv * d.D), kTile, (uint32_t)d.D,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -510,6 +518,12 @@ sage_status sage_debug_bounded_wait(uint32_t timeout_us, void* stream) {
       cudaSuccess)
     return SAGE_ERR_CUDA;
   return sage_last_device_error(stream);
+}
+
+sage_status sage_debug_kv_quant_two_pass(int32_t on) {
+  if (on != 0 && on != 1) return SAGE_ERR_INVALID_ARG;
+  g_kv_two_pass = on;
+  return SAGE_OK;
 }
 
 sage_status sage_debug_exp2_poly(const float* x, float* y, int32_t n, void* stream) {

@@ -30,6 +30,12 @@ struct QuantArgs {
   double* ksum;     // [B,Hkv,D] fp64 column sums of K
   unsigned* vamax;  // [B,Hkv,D] bit pattern of max |V| (non-negative floats order as uints);
                     // nullptr: the statistics pass skips V (NVFP4 path)
+  // one-read K/V quantisation (kv_fused_quant_kernel); kv_sync == nullptr
+  // selects the two-pass path (statistics kernel, then the code kernels)
+  int* kv_sync;          // [1 + 2 B Hkv] ints: ticket counter, tiles published per
+                         // (head, K|V) group
+  size_t kv_zero_bytes;  // bytes from ksum through the end of kv_sync (consecutive in
+                         // the workspace), zeroed before the one-read kernel
   // NVFP4 path (E2M1 codes two per byte, low nibble first; 1 KB scale blocks
   // per 128-row tile in the tcgen05 scale-factor order)
   uint8_t* q4;   // [B,Hq,Np,D/2]

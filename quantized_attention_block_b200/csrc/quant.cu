@@ -228,68 +228,19 @@ __device__ __forceinline__ void lds8(const T* p, float (&x)[8]) {
   }
 }
 
-// Q (BQ-row blocks, optional block mean) or K (BQ = bk-row blocks, minus km):
-// INT8 codes of x - shift with scale amax_block / 127.
-//   IS_K = false: shift = qbar of the block when smooth_q (written to a.qbar)
-//   IS_K = true:  shift = km = mean_n K (from the fp64 column sums)
-// grid (Np/128, B*H), 256 threads, dynamic smem: 128 x D elements + 128
-//   SHIFT: the shift is applied (smooth_q for Q, smooth_k for K); otherwise it
-//   is identically zero and the block max runs on the raw 16-bit magnitudes.
+// INT8 codes of one 128-row tile in shared memory (rows past N are zero):
+// per BQ-row block, scale = max |x - shift| / 127 over the valid rows, codes
+// rint(RN((x - shift) / scale)); writes the scales (s_k or s_q) and the codes
+// (k8 or q8).  SHIFT = false: the shift is zero and the block max runs on the
+// raw 16-bit magnitudes.  Every thread of the CTA calls it.
 template <typename T, int D, int BQ, bool IS_K, bool SHIFT>
-__global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constant__ CUtensorMap tmX, QuantArgs a) {
+__device__ __forceinline__ void qk_encode(const T* sX, const float (*s_shift)[D], float* s_red, float* s_bmax,
+                                          int bh, int tile, const QuantArgs& a) {
   constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BQ, PPB = BQ / RG;
-  extern __shared__ uint8_t qk_smem_raw[];
-  T* sX = reinterpret_cast<T*>(align128(qk_smem_raw));
-  __shared__ double s_sum[kThreads][8];
-  __shared__ float s_shift[NB][D], s_red[kThreads / 32], s_bmax[NB];
-  __shared__ uint64_t bar;
-  const int bh = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
   const int valid = rows_valid(a.N, r0, kTile);
   const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
   const int Tb = IS_K ? a.Tn : a.Tm;
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x;
-    if (IS_K) {
-      const float km = a.smooth_k ? __double2float_rn(__ddiv_rn(a.ksum[(int64_t)bh * D + c], (double)a.N)) : 0.0f;
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = km;
-      if (tile == 0) a.km[(int64_t)bh * D + c] = km;
-    } else {
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = 0.0f;
-    }
-  }
-  if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh)) return;
-  if (!IS_K && SHIFT) {
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
-      double cs[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) cs[e] = 0.0;
-#pragma unroll
-      for (int p = nb * PPB; p < (nb + 1) * PPB; ++p) {
-        float x[8];
-        lds8(sX + (rg + p * RG) * D + ch * 8, x);  // rows past N are zero
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cs[e] += (double)x[e];
-      }
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
-      __syncthreads();
-      if (threadIdx.x < D) {
-        const int c = threadIdx.x;
-        double s = 0.0;
-        for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
-        const float mu = vb > 0 ? __double2float_rn(__ddiv_rn(s, (double)vb)) : 0.0f;
-        s_shift[nb][c] = mu;
-        if (vb > 0) a.qbar[((int64_t)bh * a.Tm + tile * NB + nb) * D + c] = mu;
-      }
-    }
-  }
-  __syncthreads();
   // block max of |x - shift| over the valid rows
   float bm[NB];
   if (SHIFT) {
@@ -367,16 +318,121 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
   }
 }
 
-// V: E4M3(V / s_v[c]) per channel, transposed to [D][Np].  Each thread encodes
-// 16-token runs of one channel into a 128-byte-swizzled [D x 128] tile; one TMA
-// store writes it to v8t (the layout the attention kernel's TMA loads read).
-// grid (Np/128, B*Hkv), 256 threads, dynamic smem: D x 128 bytes + 128 x D elements
+// Q (BQ-row blocks, optional block mean) or K (BQ = bk-row blocks, minus km):
+// INT8 codes of x - shift with scale amax_block / 127.
+//   IS_K = false: shift = qbar of the block when smooth_q (written to a.qbar)
+//   IS_K = true:  shift = km = mean_n K (from the fp64 column sums)
+// grid (Np/128, B*H), 256 threads, dynamic smem: 128 x D elements + 128
+//   SHIFT: the shift is applied (smooth_q for Q, smooth_k for K); otherwise it
+//   is identically zero and the block max runs on the raw 16-bit magnitudes.
+template <typename T, int D, int BQ, bool IS_K, bool SHIFT>
+__global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constant__ CUtensorMap tmX, QuantArgs a) {
+  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BQ, PPB = BQ / RG;
+  extern __shared__ uint8_t qk_smem_raw[];
+  T* sX = reinterpret_cast<T*>(align128(qk_smem_raw));
+  __shared__ double s_sum[kThreads][8];
+  __shared__ float s_shift[NB][D], s_red[kThreads / 32], s_bmax[NB];
+  __shared__ uint64_t bar;
+  const int bh = blockIdx.y, tile = blockIdx.x;
+  const int64_t r0 = (int64_t)tile * kTile;
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    if (IS_K) {
+      const float km = a.smooth_k ? __double2float_rn(__ddiv_rn(a.ksum[(int64_t)bh * D + c], (double)a.N)) : 0.0f;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = km;
+      if (tile == 0) a.km[(int64_t)bh * D + c] = km;
+    } else {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = 0.0f;
+    }
+  }
+  if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh)) return;
+  if (!IS_K && SHIFT) {
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
+      double cs[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+      for (int p = nb * PPB; p < (nb + 1) * PPB; ++p) {
+        float x[8];
+        lds8(sX + (rg + p * RG) * D + ch * 8, x);  // rows past N are zero
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cs[e] += (double)x[e];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
+      __syncthreads();
+      if (threadIdx.x < D) {
+        const int c = threadIdx.x;
+        double s = 0.0;
+        for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
+        const float mu = vb > 0 ? __double2float_rn(__ddiv_rn(s, (double)vb)) : 0.0f;
+        s_shift[nb][c] = mu;
+        if (vb > 0) a.qbar[((int64_t)bh * a.Tm + tile * NB + nb) * D + c] = mu;
+      }
+    }
+  }
+  __syncthreads();
+  qk_encode<T, D, BQ, IS_K, SHIFT>(sX, s_shift, s_red, s_bmax, bh, tile, a);
+}
+
+// E4M3 codes of one 128-token V tile in shared memory (rows past N are zero),
+// V / s_v[c] per channel, transposed: each thread encodes 16-token runs of one
+// channel into registers; after a CTA barrier they are written as a
+// 128-byte-swizzled [D x 128] tile at sVt (1024-byte aligned; it may overlay
+// the V tile, which is consumed by then), and one TMA store writes that to
+// v8t (the layout the attention kernel's TMA loads read).  Every thread of
+// the CTA calls it; s_sv holds s_v of the head.
+template <typename T, int D>
+__device__ __forceinline__ void v_encode(const T* sV, uint8_t* sVt, const float* s_sv, const CUtensorMap* tmVt,
+                                         int tile, int bg) {
+  constexpr int TG = kThreads / D;       // token groups
+  constexpr int RUNS = kTile / 16 / TG;  // 16-token runs per thread
+  const int c = threadIdx.x % D, tg = threadIdx.x / D;
+  const float sv = s_sv[c];
+  const float rv = sv == 0.0f ? 0.0f : __frcp_rn(sv);
+  uint4 codes[RUNS];
+#pragma unroll
+  for (int q = 0; q < RUNS; ++q) {
+    const int run = tg * RUNS + q;
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 16; u += 4) {
+      float f[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f[e] = to_float(sV[(run * 16 + u + e) * D + c]);
+      w[u / 4] = sv == 0.0f ? 0u : quant_e4m3x2(f[0], f[1], sv, rv) | (quant_e4m3x2(f[2], f[3], sv, rv) << 16);
+    }
+    codes[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  __syncthreads();  // every thread has read the V tile
+#pragma unroll
+  for (int q = 0; q < RUNS; ++q) {
+    const int run = tg * RUNS + q;
+    *reinterpret_cast<uint4*>(sVt + c * kTile + ((run ^ (c & 7)) << 4)) = codes[q];
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tma_store_2d(tmVt, sVt, tile * kTile, bg * D);
+    tma_store_commit_and_wait_read();
+  }
+}
+
+// V: E4M3(V / s_v[c]) per channel, transposed to [D][Np] (v_encode; the codes
+// overlay the tile).  grid (Np/128, B*Hkv), 256 threads, dynamic smem:
+// 128 x D elements + 1024
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
     v_quant_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmVt, QuantArgs a) {
   extern __shared__ uint8_t v_smem_raw[];
   uint8_t* sVt = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(v_smem_raw) + 1023) & ~uintptr_t(1023));
-  T* sV = reinterpret_cast<T*>(sVt + D * kTile);
+  T* sV = reinterpret_cast<T*>(sVt);
   __shared__ float s_sv[D];
   __shared__ uint64_t bar;
   const int bg = blockIdx.y, tile = blockIdx.x;
@@ -388,30 +444,169 @@ __global__ void __launch_bounds__(kThreads)
     if (tile == 0) a.s_v[(int64_t)bg * D + c] = sv;
   }
   if (!load_tile<T, D>(sV, &tmX, &bar, (int)r0, bg)) return;
-  constexpr int TG = kThreads / D;       // token groups
-  constexpr int RUNS = kTile / 16 / TG;  // 16-token runs per thread
-  const int c = threadIdx.x % D, tg = threadIdx.x / D;
-  const float sv = s_sv[c];
-  const float rv = sv == 0.0f ? 0.0f : __frcp_rn(sv);
-#pragma unroll
-  for (int q = 0; q < RUNS; ++q) {
-    const int run = tg * RUNS + q;
-    uint32_t w[4];
-#pragma unroll
-    for (int u = 0; u < 16; u += 4) {
-      float f[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) f[e] = to_float(sV[(run * 16 + u + e) * D + c]);  // rows past N are zero
-      w[u / 4] = sv == 0.0f ? 0u : quant_e4m3x2(f[0], f[1], sv, rv) | (quant_e4m3x2(f[2], f[3], sv, rv) << 16);
+  v_encode<T, D>(sV, sVt, s_sv, &tmVt, tile, bg);
+}
+
+// ---------------------------------------------------------------------------
+// One-read K and V quantisation.  smooth K needs the mean of K over all N
+// tokens and psi_V the max |V| of each channel over all N, so the two-pass
+// path reads K and V twice (statistics, then codes).  Here a CTA loads one
+// 128-token tile of K or V once, adds the tile's column sums (fp64) or
+// column max |V| into its head's totals (the atomics of the statistics pass:
+// fp64 sums of 16-bit inputs do not round, so the order does not matter),
+// counts itself as published, and keeps the tile in shared memory until all
+// tiles of its (head, K|V) group have published; then it reads km or s_v
+// from the totals and writes its codes.
+//
+// Work items are handed out by ticket (one atomic increment per CTA), so
+// tickets follow the order in which CTAs start: every lower ticket belongs to
+// a CTA that is running or has finished.  A group's tiles hold consecutive
+// tickets and wait only on each other, so every wait ends as long as one
+// group fits in the CTAs resident at once (the launcher checks
+// tiles <= resident / 2 and otherwise takes the two-pass path).
+// Ticket t: group g = t / tiles = 2 (b Hkv + h) + (0: K, 1: V), tile t % tiles.
+// grid (2 tiles B Hkv), 256 threads, dynamic smem: 128 x D elements + 1024
+// (the V codes overlay the tile)
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait (one thread) for *counter >= target; false (and the timeout
+// error recorded) when the limit ran out.
+__device__ __noinline__ bool wait_count(const int* counter, int target) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = g_wait_limit_ns;
+  while (true) {
+    __nanosleep(100);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if (globaltimer_ns() - t0 > limit) {
+      record_error(kDevErrTimeout);
+      return false;
     }
-    *reinterpret_cast<uint4*>(sVt + c * kTile + ((run ^ (c & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  fence_proxy_async_smem();
+}
+
+template <typename T>
+__device__ __forceinline__ float half_bits_to_float(uint32_t m16) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+    return __uint_as_float(m16 << 16);
+  else
+    return __half2float(__ushort_as_half((unsigned short)m16));
+}
+
+template <typename T, int D, int BK, bool SMOOTH_K>
+__global__ void __launch_bounds__(kThreads)
+    kv_fused_quant_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const __grid_constant__ CUtensorMap tmVt, QuantArgs a) {
+  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BK, NW = kThreads / 32;
+  extern __shared__ uint8_t kvf_smem_raw[];
+  uint8_t* sVt = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(kvf_smem_raw) + 1023) & ~uintptr_t(1023));
+  T* sX = reinterpret_cast<T*>(sVt);
+  __shared__ double s_pk[NW * D];                       // per-warp column sums (K group)
+  unsigned* s_pv = reinterpret_cast<unsigned*>(s_pk);  // per-warp column max |V| bits (V group)
+  __shared__ float s_shift[NB][D], s_red[NW], s_bmax[NB];
+  __shared__ uint64_t bar;
+  __shared__ int s_item, s_ok;
+  const int tiles = (int)(a.Np / kTile);
+  int* published = a.kv_sync + 1;
+  if (threadIdx.x == 0) s_item = atomicAdd(a.kv_sync, 1);
+  __syncthreads();
+  const int grp = s_item / tiles, tile = s_item % tiles;
+  const int bh = grp >> 1;
+  const bool is_v = (grp & 1) != 0;
+  if (!load_tile<T, D>(sX, is_v ? &tmV : &tmK, &bar, tile * kTile, bh)) return;
+  if (!is_v && !SMOOTH_K) {  // km = 0: nothing to wait for
+    if (tile == 0 && threadIdx.x < D) a.km[(int64_t)bh * D + threadIdx.x] = 0.0f;
+    qk_encode<T, D, BK, true, false>(sX, s_shift, s_red, s_bmax, bh, tile, a);
+    return;
+  }
+  // ---- this tile's column statistics (rows past N are zero and change nothing)
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (!is_v) {
+    double cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      float x[8];
+      lds8(sX + (rg + p * RG) * D + ch * 8, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] += (double)x[e];
+    }
+    // lanes l, l + CH, ... of a warp hold the same channels
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], o);
+    if (lane < CH)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_pk[warp * D + ch * 8 + e] = cs[e];
+  } else {
+    // max |v| on the bit patterns (non-negative 16-bit floats order as integers)
+    uint32_t mv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const uint4 u = *reinterpret_cast<const uint4*>(sX + (rg + p * RG) * D + ch * 8);
+      mv[0] = __vmaxu2(mv[0], u.x & 0x7FFF7FFFu);
+      mv[1] = __vmaxu2(mv[1], u.y & 0x7FFF7FFFu);
+      mv[2] = __vmaxu2(mv[2], u.z & 0x7FFF7FFFu);
+      mv[3] = __vmaxu2(mv[3], u.w & 0x7FFF7FFFu);
+    }
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mv[i] = __vmaxu2(mv[i], __shfl_xor_sync(0xffffffffu, mv[i], o));
+    if (lane < CH)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        s_pv[warp * D + ch * 8 + 2 * i] = __float_as_uint(half_bits_to_float<T>(mv[i] & 0xFFFFu));
+        s_pv[warp * D + ch * 8 + 2 * i + 1] = __float_as_uint(half_bits_to_float<T>(mv[i] >> 16));
+      }
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    if (!is_v) {
+      double s = 0.0;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) s += s_pk[w * D + c];
+      atomicAdd(a.ksum + (int64_t)bh * D + c, s);
+    } else {
+      unsigned m = 0u;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) m = max(m, s_pv[w * D + c]);
+      atomicMax(a.vamax + (int64_t)bh * D + c, m);
+    }
+    __threadfence();
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
-    tma_store_2d(&tmVt, sVt, (int)r0, bg * D);
-    tma_store_commit_and_wait_read();
+    atomicAdd(published + grp, 1);
+    s_ok = wait_count(published + grp, tiles) ? 1 : 0;  // every tile of the group added its part
   }
+  __syncthreads();
+  if (!s_ok) return;  // timeout recorded; the codes of this tile are not written
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    if (!is_v) {
+      const float km = __double2float_rn(__ddiv_rn(__ldcg(a.ksum + (int64_t)bh * D + c), (double)a.N));
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = km;
+      if (tile == 0) a.km[(int64_t)bh * D + c] = km;
+    } else {
+      const float sv = __fdiv_rn(__uint_as_float(__ldcg(a.vamax + (int64_t)bh * D + c)), 448.0f);
+      s_shift[0][c] = sv;
+      if (tile == 0) a.s_v[(int64_t)bh * D + c] = sv;
+    }
+  }
+  __syncthreads();
+  if (!is_v)
+    qk_encode<T, D, BK, true, SMOOTH_K>(sX, s_shift, s_red, s_bmax, bh, tile, a);
+  else
+    v_encode<T, D>(sX, sVt, s_shift[0], &tmVt, tile, bh);
 }
 
 // ---------------------------------------------------------------------------
@@ -493,28 +688,54 @@ __global__ void __launch_bounds__(kThreads) delta_s_kernel(QuantArgs a) {
   }
 }
 
+// The one-read K/V kernel for (bk, smooth_k), or nullptr if a (head, K|V)
+// group of `tiles` CTAs might not fit in half of the CTAs resident at once
+// (then the two-pass path runs).  head_dim 64 also takes the two-pass path:
+// a 16 KB tile per CTA does not amortise the ticket, fence and wait (measured
+// 2.5 % slower than two passes on B=2, H=48, N=17776; head_dim 128: 12 % and
+// 6 % faster on N=4096 and N=32768).
+template <typename T, int D>
+void (*kv_fused_kernel(const QuantArgs& a, int tiles, int smem))(CUtensorMap, CUtensorMap, CUtensorMap, QuantArgs) {
+  if (D != 128) return nullptr;
+  auto kf = a.bk == 64 ? (a.smooth_k ? kv_fused_quant_kernel<T, D, 64, true> : kv_fused_quant_kernel<T, D, 64, false>)
+                       : (a.smooth_k ? kv_fused_quant_kernel<T, D, 128, true> : kv_fused_quant_kernel<T, D, 128, false>);
+  if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return nullptr;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kf, kThreads, smem) != cudaSuccess)
+    return nullptr;
+  return (int64_t)tiles * 2 <= (int64_t)sms * per_sm ? kf : nullptr;
+}
+
 template <typename T, int D>
 cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t st) {
   cudaError_t e;
   const int BHkv = a.B * a.Hkv, BHq = a.B * a.Hq;
   const int tiles = (int)(a.Np / kTile);
-  if (a.smooth_k) {
-    e = cudaMemsetAsync(a.ksum, 0, sizeof(double) * (size_t)BHkv * D, st);
+  const int smem_kvf = kTile * D * (int)sizeof(T) + 1024;
+  auto kf = a.kv_sync ? kv_fused_kernel<T, D>(a, tiles, smem_kvf) : nullptr;
+  if (kf) {
+    // ksum, vamax and kv_sync are consecutive in the workspace: one memset
+    e = cudaMemsetAsync(a.ksum, 0, a.kv_zero_bytes, st);
     if (e != cudaSuccess) return e;
+    kf<<<dim3(2 * tiles * BHkv), kThreads, smem_kvf, st>>>(m.k, m.v, m.vt, a);
   }
-  e = cudaMemsetAsync(a.vamax, 0, sizeof(unsigned) * (size_t)BHkv * D, st);
-  if (e != cudaSuccess) return e;
-  kv_stats_kernel<T, D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(a);
   const int smem_qk = kTile * D * (int)sizeof(T) + 128;
-  {
+  if (!kf) {  // two passes: column statistics, then the K and V codes
+    if (a.smooth_k) {
+      e = cudaMemsetAsync(a.ksum, 0, sizeof(double) * (size_t)BHkv * D, st);
+      if (e != cudaSuccess) return e;
+    }
+    e = cudaMemsetAsync(a.vamax, 0, sizeof(unsigned) * (size_t)BHkv * D, st);
+    if (e != cudaSuccess) return e;
+    kv_stats_kernel<T, D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(a);
     auto kq = a.bk == 64 ? (a.smooth_k ? qk_quant_kernel<T, D, 64, true, true> : qk_quant_kernel<T, D, 64, true, false>)
                          : (a.smooth_k ? qk_quant_kernel<T, D, 128, true, true> : qk_quant_kernel<T, D, 128, true, false>);
     e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_qk);
     if (e != cudaSuccess) return e;
     kq<<<dim3(tiles, BHkv), kThreads, smem_qk, st>>>(m.k, a);
-  }
-  {
-    const int smem = D * kTile + kTile * D * (int)sizeof(T) + 1024;
+    const int smem = kTile * D * (int)sizeof(T) + 1024;
     e = cudaFuncSetAttribute(v_quant_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     v_quant_kernel<T, D><<<dim3(tiles, BHkv), kThreads, smem, st>>>(m.v, m.vt, a);

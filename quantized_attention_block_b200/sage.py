@@ -27,7 +27,8 @@ EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized",
             "sage_debug_qk_int32", "sage_last_device_error", "sage_debug_bounded_wait",
             "sage_status_string", "sage_attn_fwd_noalloc", "sage_debug_f8_accum_probe",
             "sage_nvfp4_workspace_bytes", "sage_quant_nvfp4", "sage_attn_fwd_nvfp4_quantized",
-            "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4", "sage_debug_exp2_poly")
+            "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4", "sage_debug_exp2_poly",
+            "sage_debug_kv_quant_two_pass")
 
 
 class SageError(RuntimeError):
@@ -90,6 +91,7 @@ def lib() -> ctypes.CDLL:
         L.sage_attn_fwd_nvfp4.argtypes = [vp, vp, vp, vp, P, vp, ctypes.c_size_t, vp]
         L.sage_debug_qk_nvfp4.argtypes = [F, P, i32, i32, i32, i32, vp, vp]
         L.sage_debug_exp2_poly.argtypes, L.sage_debug_exp2_poly.restype = [vp, vp, i32, vp], ctypes.c_int
+        L.sage_debug_kv_quant_two_pass.argtypes, L.sage_debug_kv_quant_two_pass.restype = [i32], ctypes.c_int
         for n in ("sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd", "sage_debug_qk_int32",
                   "sage_last_device_error", "sage_debug_bounded_wait", "sage_quant_nvfp4",
                   "sage_attn_fwd_nvfp4_quantized", "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4"):
@@ -269,6 +271,11 @@ def sage_debug_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
     y = torch.empty_like(x)
     _check(lib().sage_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "sage_debug_exp2_poly")
     return y
+
+
+def sage_debug_kv_quant_two_pass(on: bool) -> None:
+    """Force (True) or release (False) the two-pass K/V quantisation path in this process."""
+    _check(lib().sage_debug_kv_quant_two_pass(1 if on else 0), "sage_debug_kv_quant_two_pass")
 
 
 def nvfp4_view_tensors(view: SageNvfp4View, p: SageParams, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:

@@ -43,6 +43,30 @@ def test_quant_bit_exact(name):
     assert not bad, bad
 
 
+@pytest.mark.parametrize("name", list(SMALL) + list(EDGE))
+def test_one_read_kv_quant_equals_two_pass(name):
+    """The one-read K/V kernel (each tile waits in shared memory for its head's
+    km / s_v) and the two-pass path (statistics kernel first) write the same
+    bytes: codes, scales, km, qbar and delta_S."""
+    w = {**SMALL, **EDGE}[name]
+    q, k, v = W.make_qkv(w)
+    p, ws1, view1, _ = gpu_quant(w, q, k, v)
+    assert sage.sage_last_device_error() == 0
+    sage.sage_debug_kv_quant_two_pass(True)
+    try:
+        _, ws2, view2, _ = gpu_quant(w, q, k, v)
+    finally:
+        sage.sage_debug_kv_quant_two_pass(False)
+    assert sage.sage_last_device_error() == 0
+    t1, t2 = sage.view_tensors(view1, p, ws1), sage.view_tensors(view2, p, ws2)
+    assert t1.keys() == t2.keys()
+    for key in t1:
+        a = t1[key].contiguous().cpu().numpy()
+        b = t2[key].contiguous().cpu().numpy()
+        assert a.shape == b.shape, key
+        np.testing.assert_array_equal(a.reshape(-1).view(np.uint8), b.reshape(-1).view(np.uint8), err_msg=key)
+
+
 @pytest.mark.parametrize("name", ["tiny", "prefill", "video", "gqa"])
 def test_qk_int32_tiles_bit_exact(name):
     w = SMALL[name]
