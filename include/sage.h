@@ -282,6 +282,15 @@ SAGE_API sage_status sage_debug_qk_nvfp4(const sage_nvfp4_view *view, const sage
 SAGE_API sage_status sage_debug_exp2_poly(const float *x, float *y, int32_t n, void *stream);
 
 /*
+ * Number of kernels sage_quant_qkv enqueues for p on the current device (not
+ * counting memsets): 2 with the one-read K/V kernel (K and V, then Q), 4 with
+ * the two-pass path (K/V statistics, K, V, Q); +1 with smooth_q (delta_S).
+ * *n is written on SAGE_OK.  Needs the device (the choice depends on how many
+ * CTAs it holds at once).
+ */
+SAGE_API sage_status sage_quant_kernel_count(const sage_params *p, int32_t *n);
+
+/*
  * Test hook: on = 1 makes sage_quant_qkv (and the calls built on it) take the
  * two-pass K/V path (statistics kernel, then the code kernels) in this
  * process; on = 0 restores the default choice.  Not thread-safe with

@@ -520,6 +520,29 @@ sage_status sage_debug_bounded_wait(uint32_t timeout_us, void* stream) {
   return sage_last_device_error(stream);
 }
 
+sage_status sage_quant_kernel_count(const sage_params* p, int32_t* n) {
+  Dims d;
+  sage_status s = check_params(p, &d);
+  if (s != SAGE_OK) return s;
+  if (!n) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_arch()) != SAGE_OK) return s;
+  QuantArgs a{};
+  a.B = (int)d.B;
+  a.Hq = (int)d.Hq;
+  a.Hkv = (int)d.Hkv;
+  a.N = (int)d.N;
+  a.D = (int)d.D;
+  a.Np = d.Np;
+  a.Tm = (int)d.Tm;
+  a.Tn = (int)d.Tn;
+  a.bq = p->bq;
+  a.bk = p->bk;
+  a.smooth_k = p->smooth_k;
+  a.smooth_q = p->smooth_q;
+  *n = quant_kernel_count(a, p->dtype == SAGE_FP16, g_kv_two_pass == 0);
+  return SAGE_OK;
+}
+
 sage_status sage_debug_kv_quant_two_pass(int32_t on) {
   if (on != 0 && on != 1) return SAGE_ERR_INVALID_ARG;
   g_kv_two_pass = on;

@@ -76,6 +76,10 @@ struct QuantMaps {
 };
 
 // launchers (defined in the .cu files)
+// kernels (not counting memsets) that launch_quant enqueues for a's sizes and
+// flags (the one-read K/V path if allowed and it fits the current device,
+// else the two-pass path)
+int quant_kernel_count(const QuantArgs& a, int is_fp16, bool allow_one_read);
 cudaError_t launch_quant(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st);
 cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, cudaStream_t st);

@@ -756,7 +756,22 @@ cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t 
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+int quant_kernel_count_t(const QuantArgs& a, bool allow_one_read) {
+  const int tiles = (int)(a.Np / kTile);
+  const bool one_read = allow_one_read && kv_fused_kernel<T, D>(a, tiles, kTile * D * (int)sizeof(T) + 1024);
+  return (one_read ? 2 : 4) + (a.smooth_q ? 1 : 0);
+}
+
 }  // namespace
+
+int quant_kernel_count(const QuantArgs& a, int is_fp16, bool allow_one_read) {
+  if (is_fp16)
+    return a.D == 128 ? quant_kernel_count_t<__half, 128>(a, allow_one_read)
+                      : quant_kernel_count_t<__half, 64>(a, allow_one_read);
+  return a.D == 128 ? quant_kernel_count_t<__nv_bfloat16, 128>(a, allow_one_read)
+                    : quant_kernel_count_t<__nv_bfloat16, 64>(a, allow_one_read);
+}
 
 cudaError_t launch_quant(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st) {
   if (is_fp16) return a.D == 128 ? launch_quant_t<__half, 128>(a, m, st) : launch_quant_t<__half, 64>(a, m, st);

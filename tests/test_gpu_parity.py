@@ -67,6 +67,22 @@ def test_one_read_kv_quant_equals_two_pass(name):
         np.testing.assert_array_equal(a.reshape(-1).view(np.uint8), b.reshape(-1).view(np.uint8), err_msg=key)
 
 
+def test_quant_kernel_count_follows_the_path():
+    """head_dim 128 takes the one-read K/V kernel (2 kernels + delta_S), head_dim
+    64 and the forced two-pass path 4 (+ delta_S)."""
+    for name, one_read in (("prefill", True), ("gqa", True), ("video", False)):
+        w = W.get(name)
+        p = sage.SageParams(w.B, w.Hq, w.Hkv, w.N, w.d, 0, int(w.causal), float(w.sm_scale or 0.0),
+                            int(w.smooth_k), int(w.smooth_q), w.bq, w.bk, 0)
+        extra = 1 if w.smooth_q else 0
+        assert sage.sage_quant_kernel_count(p) == (2 if one_read else 4) + extra, name
+        sage.sage_debug_kv_quant_two_pass(True)
+        try:
+            assert sage.sage_quant_kernel_count(p) == 4 + extra, name
+        finally:
+            sage.sage_debug_kv_quant_two_pass(False)
+
+
 @pytest.mark.parametrize("name", ["tiny", "prefill", "video", "gqa"])
 def test_qk_int32_tiles_bit_exact(name):
     w = SMALL[name]
