@@ -6,7 +6,7 @@
 //   smooth Q:  qbar_i = mean of Q block i,  Q_i - qbar_i
 //   psi_Q/psi_K: per-block INT8, scale = amax / 127, code = rint(x / scale)
 //   psi_V:     per-channel FP8 E4M3, scale = amax / 448
-//   GEMV:      delta_S[i, j] = qbar_i . gamma(K_j)
+//   GEMV:      delta_S[i, j] = qbar_i . gamma(K_j)   (tcgen05 TF32, 3-term split)
 // Bit-exactness with the plain definitions: column sums are accumulated in
 // fp64 (the partial sums of bf16/fp16 inputs are exact, so the order does
 // not matter), divided in fp64 and rounded once to fp32; every division of
@@ -327,7 +327,7 @@ __device__ __forceinline__ void qk_encode(const T* sX, const float (*s_shift)[D]
 //   is identically zero and the block max runs on the raw 16-bit magnitudes.
 template <typename T, int D, int BQ, bool IS_K, bool SHIFT>
 __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constant__ CUtensorMap tmX, QuantArgs a) {
-  constexpr int CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BQ, PPB = BQ / RG;
+  constexpr int CH = D / 8, RG = kThreads / CH, NB = kTile / BQ, PPB = BQ / RG;
   extern __shared__ uint8_t qk_smem_raw[];
   T* sX = reinterpret_cast<T*>(align128(qk_smem_raw));
   __shared__ double s_sum[kThreads][8];
@@ -610,82 +610,199 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Pass 3 (smooth Q): delta_S[b,h,i,j] = sum_c qbar[i,c] * gamma(K)[j,c] for one
-// 128-key tile and every Q block i.  fp32 accumulation in channel order.
-// gamma(K)^T [D][128] and 32-block chunks of qbar^T [D][32] sit in shared
-// memory; each thread accumulates a 4-block x 4-key tile (two f32x2 FMAs per
-// block and channel), so every shared load feeds eight FMAs.
-// grid (Np/128, B*Hq), 256 threads; dynamic smem: (D*128 + D*32) floats
-constexpr int kDsBlocks = 32;  // Q blocks per chunk
+// delta_S on the tensor cores.  Per (b, h) and 128-key tile j:
+//   delta_S^T[key, i] = sum_c gamma(K)[key, c] qbar[i, c]
+// is a [128 x d] x [d x Tm] contraction, so it runs as tcgen05.mma kind::tf32
+// with the keys as M (the accumulator's TMEM lanes) and the Q blocks as N.
+// TF32 keeps 10 of fp32's 23 mantissa bits, so each operand is split exactly
+// into x = hi + lo (hi: x with the low 13 mantissa bits cleared, a TF32 value;
+// lo = x - hi, exact in fp32) and three products accumulate in FP32:
+// hi lo + lo hi first (the small terms), then hi hi; the dropped lo lo term
+// and the TF32 rounding of lo are below 2^-20 of |x y| per product.
+// The channels go through in passes of 64 (operands of 128 keys and of
+// kDsTcBlocks Q blocks, hi and lo: 104 KB, so two CTAs share an SM and one's
+// loads overlap the other's MMAs and stores); the Q blocks in chunks of
+// kDsTcBlocks (the accumulator's columns).
+// Operands in shared memory, K-major with the 128-byte swizzle: element
+// (r, c) of an R-row operand sits in 32-channel column block c / 32 (R x 128
+// bytes), row r, 16-byte unit ((c % 32) / 4) ^ (r % 8).
+// grid (Np/128, B*Hq), 256 threads; dynamic smem ds_tc_smem().  Keys past N
+// give gamma = 0, so their delta_S columns are written as zeros, like the rest
+// of the padding.
+constexpr int kDsTcBlocks = 80;  // Q blocks per chunk (MMA N <= 80)
+constexpr int kDsTcCh = 64;      // channels per pass
+
+constexpr size_t ds_tc_smem() { return (size_t)2 * (kTile + kDsTcBlocks) * kDsTcCh * 4 + 1024; }
+
+__device__ __forceinline__ uint32_t swz128_offset(int r, int c, int rows) {
+  return (uint32_t)((c >> 5) * rows * 128 + r * 128 + ((((c & 31) >> 2) ^ (r & 7)) << 4) + (c & 3) * 4);
+}
+
+// split 8 consecutive fp32 (channels c .. c + 7 of the pass, c % 8 == 0) of
+// row r into the hi / lo operands
+__device__ __forceinline__ void store_split8(uint8_t* hi, uint8_t* lo, int r, int c, int rows, const float (&x)[8]) {
+  float h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    h[e] = __uint_as_float(__float_as_uint(x[e]) & 0xFFFFE000u);
+    l[e] = __fsub_rn(x[e], h[e]);
+  }
+  const uint32_t o0 = swz128_offset(r, c, rows), o1 = swz128_offset(r, c + 4, rows);
+  *reinterpret_cast<float4*>(hi + o0) = make_float4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<float4*>(hi + o1) = make_float4(h[4], h[5], h[6], h[7]);
+  *reinterpret_cast<float4*>(lo + o0) = make_float4(l[0], l[1], l[2], l[3]);
+  *reinterpret_cast<float4*>(lo + o1) = make_float4(l[4], l[5], l[6], l[7]);
+}
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) delta_s_kernel(QuantArgs a) {
-  extern __shared__ float s_ds[];
-  float* s_gT = s_ds;               // [D][kTile]
-  float* s_qT = s_ds + D * kTile;   // [D][kDsBlocks]
+__global__ void __launch_bounds__(kThreads, 2) delta_s_tc_kernel(QuantArgs a) {
+  constexpr int NBK = kDsTcBlocks, CP = kDsTcCh, G8 = CP / 8;  // 8-channel groups per pass row
+  constexpr uint32_t kA = kTile * CP * 4, kB = NBK * CP * 4;
+  constexpr uint32_t kCols = 128;
+  static_assert(D % CP == 0 && NBK % 16 == 0 && NBK <= (int)kCols, "delta_S tile shape");
+  extern __shared__ uint8_t ds_tc_raw[];
+  uint8_t* sAh = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ds_tc_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sAl = sAh + kA;
+  uint8_t* sBh = sAl + kA;
+  uint8_t* sBl = sBh + kB;
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_slot;
   const int bh = blockIdx.y, tile = blockIdx.x;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const int bg = b * a.Hkv + h / (a.Hq / a.Hkv);
   const int64_t r0 = (int64_t)tile * kTile;
   const int valid = rows_valid(a.N, r0, kTile);
-  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, kCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&mma_bar, 1);
+    mbar_fence_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const T* K = reinterpret_cast<const T*>(a.k) + ((int64_t)bg * a.N + r0) * D;
   const float* km = a.km + (int64_t)bg * D;
-  // gamma(K) -> shared, transposed.  A warp takes 16 rows x 2 adjacent 8-channel
-  // chunks per step: 32-byte row segments from global, and its transposed
-  // stores hit each bank at most twice.
-  {
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-#pragma unroll
-    for (int it = 0; it < (kTile / 16) * (D / 16) / (kThreads / 32); ++it) {
-      const int item = warp + it * (kThreads / 32);
-      const int r = (item % (kTile / 16)) * 16 + lane / 2;
-      const int chunk = (item / (kTile / 16)) * 2 + (lane & 1);
-      float x[8];
-      if (r < valid) {
-        load8<T>(K + (r0 + r) * D + chunk * 8, x);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], km[chunk * 8 + e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.0f;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s_gT[(chunk * 8 + e) * kTile + r] = x[e];
-    }
-  }
-  const int kg = threadIdx.x % 32, bgp = threadIdx.x / 32;  // keys 4 kg.., blocks 4 bgp..
   const float* qb = a.qbar + (int64_t)bh * a.Tm * D;
-  float* out = a.dS + (int64_t)bh * a.Tm * a.Np + r0 + 4 * kg;
-  for (int i0 = 0; i0 < a.Tm; i0 += kDsBlocks) {
-    __syncthreads();  // gamma^T written / previous chunk consumed
-    for (int idx = threadIdx.x; idx < kDsBlocks * D; idx += kThreads) {
-      const int blk = idx % kDsBlocks, c = idx / kDsBlocks;  // conflict-free stores
-      s_qT[c * kDsBlocks + blk] = (i0 + blk < a.Tm) ? qb[(int64_t)(i0 + blk) * D + c] : 0.0f;
+  float* out = a.dS + (int64_t)bh * a.Tm * a.Np + r0;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int cl = (threadIdx.x % G8) * 8;  // this thread's channels within a pass (every step)
+  bool ok = true;
+  uint32_t phase = 0;
+  for (int i0 = 0; i0 < a.Tm && ok; i0 += NBK) {
+    const int nb = min(NBK, a.Tm - i0);
+    const int nbp = (nb + 15) & ~15;  // MMA N: a multiple of 16
+    const uint32_t idesc = make_idesc(/*F32*/ 1, /*TF32*/ 2, /*TF32*/ 2, kTile, nbp);
+    for (int c0 = 0; c0 < D && ok; c0 += CP, phase ^= 1u) {
+      // A = gamma(K)[:, c0 .. c0 + 64) (rows past N zero), B = qbar[i0 .., c0 ..)
+      // (rows past Tm zero); every load of the thread is issued before use
+      constexpr int ITA = kTile * G8 / kThreads, ITB = (NBK * G8 + kThreads - 1) / kThreads;
+      uint4 ka[ITA];
+      float4 qv[ITB][2];
+#pragma unroll
+      for (int it = 0; it < ITA; ++it) {
+        const int r = (threadIdx.x + it * kThreads) / G8;
+        ka[it] = r < valid ? __ldg(reinterpret_cast<const uint4*>(K + (int64_t)r * D + c0 + cl))
+                           : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int it = 0; it < ITB; ++it) {
+        const int r = (threadIdx.x + it * kThreads) / G8;
+        const float* src = qb + (int64_t)(i0 + r) * D + c0 + cl;
+        qv[it][0] = r < nb ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        qv[it][1] = r < nb ? __ldg(reinterpret_cast<const float4*>(src + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float kmc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) kmc[e] = km[c0 + cl + e];
+      // the previous pass's MMAs have read the operands (waited on below)
+#pragma unroll
+      for (int it = 0; it < ITA; ++it) {
+        const int r = (threadIdx.x + it * kThreads) / G8;
+        float x[8];
+        lds8(reinterpret_cast<const T*>(&ka[it]), x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = r < valid ? __fsub_rn(x[e], kmc[e]) : 0.0f;
+        store_split8(sAh, sAl, r, cl, kTile, x);
+      }
+#pragma unroll
+      for (int it = 0; it < ITB; ++it) {
+        const int r = (threadIdx.x + it * kThreads) / G8;
+        if (r < nbp) {
+          const float x[8] = {qv[it][0].x, qv[it][0].y, qv[it][0].z, qv[it][0].w,
+                              qv[it][1].x, qv[it][1].y, qv[it][1].z, qv[it][1].w};
+          store_split8(sBh, sBl, r, cl, NBK, x);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+        const uint32_t aH = smem_u32(sAh), aL = smem_u32(sAl), bH = smem_u32(sBh), bL = smem_u32(sBl);
+        // K step kk: 8 channels = 32 bytes inside 32-channel column block kk / 4
+#pragma unroll
+        for (int kk = 0; kk < CP / 8; ++kk) {
+          const uint32_t oa = (kk >> 2) * kTile * 128 + (kk & 3) * 32, ob = (kk >> 2) * NBK * 128 + (kk & 3) * 32;
+          mma_tf32(tmem, make_sdesc(aH + oa, 1024, kSwizzle128B), make_sdesc(bL + ob, 1024, kSwizzle128B), idesc,
+                   (c0 > 0 || kk > 0) ? 1u : 0u);
+          mma_tf32(tmem, make_sdesc(aL + oa, 1024, kSwizzle128B), make_sdesc(bH + ob, 1024, kSwizzle128B), idesc,
+                   1u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < CP / 8; ++kk) {
+          const uint32_t oa = (kk >> 2) * kTile * 128 + (kk & 3) * 32, ob = (kk >> 2) * NBK * 128 + (kk & 3) * 32;
+          mma_tf32(tmem, make_sdesc(aH + oa, 1024, kSwizzle128B), make_sdesc(bH + ob, 1024, kSwizzle128B), idesc,
+                   1u);
+        }
+        mma_commit(&mma_bar);
+      }
+      __syncwarp();
+      ok = mbar_wait_warp(&mma_bar, phase);
+      tc_fence_after();
+      ok = __syncthreads_and(ok);
     }
-    __syncthreads();
-    float2 acc[4][2];
+    if (ok) {
+      // lanes 32 quarter ..: keys; the two halves of the CTA take alternate
+      // 16-block groups
+      const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
+      const int key = quarter * 32 + lane;
+      for (int g = half; g < nbp / 16; g += 2) {
+        uint32_t v[16];
+        tmem_ld16p(tq + g * 16, v);
+        tmem_ld_wait();
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = make_float2(0.0f, 0.0f);
-#pragma unroll 4
-    for (int c = 0; c < D; ++c) {
-      const float4 q4 = *reinterpret_cast<const float4*>(s_qT + c * kDsBlocks + 4 * bgp);
-      const float4 g4 = *reinterpret_cast<const float4*>(s_gT + c * kTile + 4 * kg);
-      const float2 g01 = make_float2(g4.x, g4.y), g23 = make_float2(g4.z, g4.w);
-      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc[u][0] = ffma2(make_float2(qv[u], qv[u]), g01, acc[u][0]);
-        acc[u][1] = ffma2(make_float2(qv[u], qv[u]), g23, acc[u][1]);
+        for (int e = 0; e < 16; ++e) {
+          const int i = i0 + g * 16 + e;
+          if (i < a.Tm) out[(int64_t)i * a.Np + key] = __uint_as_float(v[e]);
+        }
       }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int blk = i0 + 4 * bgp + u;
-      if (blk < a.Tm)
-        *reinterpret_cast<float4*>(out + (int64_t)blk * a.Np) =
-            make_float4(acc[u][0].x, acc[u][0].y, acc[u][1].x, acc[u][1].y);
-    }
+    // every warp has read the accumulator before the next chunk's MMAs
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    tc_fence_after();
   }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_delta_s(const QuantArgs& a, cudaStream_t st) {
+  const int tiles = (int)(a.Np / kTile);
+  const int smem = (int)ds_tc_smem();
+  cudaError_t e = cudaFuncSetAttribute(delta_s_tc_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  delta_s_tc_kernel<T, D><<<dim3(tiles, a.B * a.Hq), kThreads, smem, st>>>(a);
+  return cudaGetLastError();
 }
 
 // The one-read K/V kernel for (bk, smooth_k), or nullptr if a (head, K|V)
@@ -748,10 +865,8 @@ cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t 
     qq<<<dim3(tiles, BHq), kThreads, smem_qk, st>>>(m.q, a);
   }
   if (a.smooth_q) {
-    const size_t smem = sizeof(float) * D * (kTile + kDsBlocks);
-    e = cudaFuncSetAttribute(delta_s_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = launch_delta_s<T, D>(a, st);
     if (e != cudaSuccess) return e;
-    delta_s_kernel<T, D><<<dim3(tiles, BHq), kThreads, smem, st>>>(a);
   }
   return cudaGetLastError();
 }

@@ -242,10 +242,8 @@ cudaError_t launch_quant_nvfp4_t(const QuantArgs& a, cudaStream_t st) {
   else
     q_quant_nvfp4_kernel<T, 128><<<dim3(tiles, BHq), kThreads, 0, st>>>(s);
   if (a.smooth_q) {
-    const size_t smem = sizeof(float) * kF4D * (kTile + kDsBlocks);
-    e = cudaFuncSetAttribute(delta_s_kernel<T, kF4D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = launch_delta_s<T, kF4D>(s, st);
     if (e != cudaSuccess) return e;
-    delta_s_kernel<T, kF4D><<<dim3(tiles, BHq), kThreads, smem, st>>>(s);
   }
   return cudaGetLastError();
 }
