@@ -699,15 +699,17 @@ __global__ void __launch_bounds__(kThreads, 2) delta_s_tc_kernel(QuantArgs a) {
     const uint32_t idesc = make_idesc(/*F32*/ 1, /*TF32*/ 2, /*TF32*/ 2, kTile, nbp);
     for (int c0 = 0; c0 < D && ok; c0 += CP, phase ^= 1u) {
       // A = gamma(K)[:, c0 .. c0 + 64) (rows past N zero), B = qbar[i0 .., c0 ..)
-      // (rows past Tm zero); every load of the thread is issued before use
+      // (rows past Tm zero); every load of the thread is issued before use.
+      // With a single pass (d = 64) A stays from the first chunk.
+      const bool load_a = D > CP || i0 == 0;
       constexpr int ITA = kTile * G8 / kThreads, ITB = (NBK * G8 + kThreads - 1) / kThreads;
       uint4 ka[ITA];
       float4 qv[ITB][2];
 #pragma unroll
       for (int it = 0; it < ITA; ++it) {
         const int r = (threadIdx.x + it * kThreads) / G8;
-        ka[it] = r < valid ? __ldg(reinterpret_cast<const uint4*>(K + (int64_t)r * D + c0 + cl))
-                           : make_uint4(0u, 0u, 0u, 0u);
+        ka[it] = (load_a && r < valid) ? __ldg(reinterpret_cast<const uint4*>(K + (int64_t)r * D + c0 + cl))
+                                       : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int it = 0; it < ITB; ++it) {
@@ -720,14 +722,16 @@ __global__ void __launch_bounds__(kThreads, 2) delta_s_tc_kernel(QuantArgs a) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) kmc[e] = km[c0 + cl + e];
       // the previous pass's MMAs have read the operands (waited on below)
+      if (load_a) {
 #pragma unroll
-      for (int it = 0; it < ITA; ++it) {
-        const int r = (threadIdx.x + it * kThreads) / G8;
-        float x[8];
-        lds8(reinterpret_cast<const T*>(&ka[it]), x);
+        for (int it = 0; it < ITA; ++it) {
+          const int r = (threadIdx.x + it * kThreads) / G8;
+          float x[8];
+          lds8(reinterpret_cast<const T*>(&ka[it]), x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = r < valid ? __fsub_rn(x[e], kmc[e]) : 0.0f;
-        store_split8(sAh, sAl, r, cl, kTile, x);
+          for (int e = 0; e < 8; ++e) x[e] = r < valid ? __fsub_rn(x[e], kmc[e]) : 0.0f;
+          store_split8(sAh, sAl, r, cl, kTile, x);
+        }
       }
 #pragma unroll
       for (int it = 0; it < ITB; ++it) {
