@@ -204,9 +204,9 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
     for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
-    # our kernels per step: the quantisation kernels (as the library reports them
-    # for the INT8 path; NVFP4: K statistics, K, V, Q [+ delta_S]) + the attention
-    n_quant = (4 + (1 if w.smooth_q else 0)) if w.nvfp4 else sage.sage_quant_kernel_count(p)
+    # our kernels per step: the quantisation kernels (as the library reports
+    # them for the path the sizes take) + the attention
+    n_quant = sage.sage_quant_nvfp4_kernel_count(p) if w.nvfp4 else sage.sage_quant_kernel_count(p)
     launches_per_step = n_quant + 1
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -291,9 +291,17 @@ SAGE_API sage_status sage_debug_exp2_poly(const float *x, float *y, int32_t n, v
 SAGE_API sage_status sage_quant_kernel_count(const sage_params *p, int32_t *n);
 
 /*
- * Test hook: on = 1 makes sage_quant_qkv (and the calls built on it) take the
- * two-pass K/V path (statistics kernel, then the code kernels) in this
- * process; on = 0 restores the default choice.  Not thread-safe with
+ * Number of kernels sage_quant_nvfp4 enqueues for p on the current device
+ * (not counting memsets): 3 with the one-read K kernel (K, V, Q), 4 with the
+ * statistics pass (K statistics, K, V, Q); +1 with smooth_q (delta_S).
+ * Argument checks as sage_quant_nvfp4 (head_dim 128 only).
+ */
+SAGE_API sage_status sage_quant_nvfp4_kernel_count(const sage_params *p, int32_t *n);
+
+/*
+ * Test hook: on = 1 makes sage_quant_qkv and sage_quant_nvfp4 (and the calls
+ * built on them) take the two-pass K/V path (statistics kernel, then the code
+ * kernels) in this process; on = 0 restores the default choice.  Not thread-safe with
  * concurrent sage_quant_qkv calls.  SAGE_ERR_INVALID_ARG for other values.
  */
 SAGE_API sage_status sage_debug_kv_quant_two_pass(int32_t on);

@@ -200,7 +200,7 @@ sage_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_
 
 // ---------------------------------------------------------------- NVFP4 layout
 struct LayoutF4 {
-  size_t q4, k4, v4t, sfq, sfk, sfv, km, ksum, qbar, dS, total;
+  size_t q4, k4, v4t, sfq, sfk, sfv, km, ksum, kv_sync, kv_sync_end, qbar, dS, total;
 };
 
 LayoutF4 make_layout_f4(const sage_params* p, const Dims& d) {
@@ -219,7 +219,10 @@ LayoutF4 make_layout_f4(const sage_params* p, const Dims& d) {
   L.sfk = take((size_t)(d.B * d.Hkv) * tiles * 1024);
   L.sfv = take((size_t)(d.B * d.Hkv) * tiles * 1024);
   L.km = take(4 * (size_t)(d.B * d.Hkv * d.D));
+  // ksum, kv_sync consecutive: the one-read K kernel zeroes them with one memset
   L.ksum = take(8 * (size_t)(d.B * d.Hkv * d.D));
+  L.kv_sync = take(4 * (size_t)(1 + d.B * d.Hkv));
+  L.kv_sync_end = L.kv_sync + 4 * (size_t)(1 + d.B * d.Hkv);
   if (p->smooth_q) {
     L.qbar = take(4 * (size_t)(d.B * d.Hq * d.Tm * d.D));
     L.dS = take(4 * (size_t)(d.B * d.Hq * d.Tm * d.Np));
@@ -440,7 +443,15 @@ sage_status sage_quant_nvfp4(const void* q, const void* k, const void* v, const 
   a.sfq = view->sfq;
   a.sfk = view->sfk;
   a.sfv = view->sfv;
-  return from_cuda(launch_quant_nvfp4(a, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
+  a.kv_sync = g_kv_two_pass ? nullptr : reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + L.kv_sync);
+  a.kv_zero_bytes = L.kv_sync_end - L.ksum;
+  QuantMaps m;
+  if (!map_3d_input(&m.q, q, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hq)) ||
+      !map_3d_input(&m.k, k, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)) ||
+      !map_3d_input(&m.v, v, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)))
+    return SAGE_ERR_CUDA;
+  m.vt = m.v;  // unused on this path
+  return from_cuda(launch_quant_nvfp4(a, m, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status sage_attn_fwd_nvfp4_quantized(const sage_nvfp4_view* view, void* o, const sage_params* p,
@@ -540,6 +551,29 @@ sage_status sage_quant_kernel_count(const sage_params* p, int32_t* n) {
   a.smooth_k = p->smooth_k;
   a.smooth_q = p->smooth_q;
   *n = quant_kernel_count(a, p->dtype == SAGE_FP16, g_kv_two_pass == 0);
+  return SAGE_OK;
+}
+
+sage_status sage_quant_nvfp4_kernel_count(const sage_params* p, int32_t* n) {
+  Dims d;
+  sage_status s = check_params_f4(p, &d);
+  if (s != SAGE_OK) return s;
+  if (!n) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_arch()) != SAGE_OK) return s;
+  QuantArgs a{};
+  a.B = (int)d.B;
+  a.Hq = (int)d.Hq;
+  a.Hkv = (int)d.Hkv;
+  a.N = (int)d.N;
+  a.D = (int)d.D;
+  a.Np = d.Np;
+  a.Tm = (int)d.Tm;
+  a.Tn = (int)d.Tn;
+  a.bq = p->bq;
+  a.bk = p->bk;
+  a.smooth_k = p->smooth_k;
+  a.smooth_q = p->smooth_q;
+  *n = quant_nvfp4_kernel_count(a, p->dtype == SAGE_FP16, g_kv_two_pass == 0);
   return SAGE_OK;
 }
 

@@ -32,8 +32,9 @@ struct QuantArgs {
                     // nullptr: the statistics pass skips V (NVFP4 path)
   // one-read K/V quantisation (kv_fused_quant_kernel); kv_sync == nullptr
   // selects the two-pass path (statistics kernel, then the code kernels)
-  int* kv_sync;          // [1 + 2 B Hkv] ints: ticket counter, tiles published per
-                         // (head, K|V) group
+  int* kv_sync;          // ticket counter, then tiles published per group: [1 + 2 B Hkv]
+                         // ints on the INT8 path ((head, K|V) groups), [1 + B Hkv] on the
+                         // NVFP4 path (K only)
   size_t kv_zero_bytes;  // bytes from ksum through the end of kv_sync (consecutive in
                          // the workspace), zeroed before the one-read kernel
   // NVFP4 path (E2M1 codes two per byte, low nibble first; 1 KB scale blocks
@@ -87,7 +88,9 @@ cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUt
 cudaError_t launch_bounded_wait_probe(cudaStream_t st);
 cudaError_t launch_exp2_poly_probe(const float* x, float* y, int n, cudaStream_t st);
 cudaError_t launch_f8_accum_probe(float* out, cudaStream_t st);
-cudaError_t launch_quant_nvfp4(const QuantArgs& a, int is_fp16, cudaStream_t st);
+cudaError_t launch_quant_nvfp4(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st);
+// kernels (not counting memsets) that launch_quant_nvfp4 enqueues for a's sizes and flags
+int quant_nvfp4_kernel_count(const QuantArgs& a, int is_fp16, bool allow_one_read);
 cudaError_t launch_attn_nvfp4(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                               const CUtensorMap& tmV, cudaStream_t st);
 cudaError_t launch_qk_probe_nvfp4(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,

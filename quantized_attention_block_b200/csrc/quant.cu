@@ -318,6 +318,44 @@ __device__ __forceinline__ void qk_encode(const T* sX, const float (*s_shift)[D]
   }
 }
 
+// smooth Q: the column means of each BQ-row block of a 128-row tile in shared
+// memory (rows past N are zero): fp64 sums over the block, one fp64 division
+// by its number of valid rows, one rounding to fp32 -> s_mean[nb][c], also
+// written to qbar (when the block has rows).  Every thread of the CTA calls it.
+template <typename T, int D, int BQ>
+__device__ __forceinline__ void block_means(const T* sX, double (*s_sum)[8], float (*s_mean)[D], int bh, int tile,
+                                            const QuantArgs& a) {
+  constexpr int CH = D / 8, RG = kThreads / CH, NB = kTile / BQ, PPB = BQ / RG;
+  const int64_t r0 = (int64_t)tile * kTile;
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
+    double cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+    for (int p = nb * PPB; p < (nb + 1) * PPB; ++p) {
+      float x[8];
+      lds8(sX + (rg + p * RG) * D + ch * 8, x);  // rows past N are zero
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] += (double)x[e];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      const int c = threadIdx.x;
+      double s = 0.0;
+      for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
+      const float mu = vb > 0 ? __double2float_rn(__ddiv_rn(s, (double)vb)) : 0.0f;
+      s_mean[nb][c] = mu;
+      if (vb > 0) a.qbar[((int64_t)bh * a.Tm + tile * NB + nb) * D + c] = mu;
+    }
+  }
+}
+
 // Q (BQ-row blocks, optional block mean) or K (BQ = bk-row blocks, minus km):
 // INT8 codes of x - shift with scale amax_block / 127.
 //   IS_K = false: shift = qbar of the block when smooth_q (written to a.qbar)
@@ -327,7 +365,7 @@ __device__ __forceinline__ void qk_encode(const T* sX, const float (*s_shift)[D]
 //   is identically zero and the block max runs on the raw 16-bit magnitudes.
 template <typename T, int D, int BQ, bool IS_K, bool SHIFT>
 __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constant__ CUtensorMap tmX, QuantArgs a) {
-  constexpr int CH = D / 8, RG = kThreads / CH, NB = kTile / BQ, PPB = BQ / RG;
+  constexpr int NB = kTile / BQ;
   extern __shared__ uint8_t qk_smem_raw[];
   T* sX = reinterpret_cast<T*>(align128(qk_smem_raw));
   __shared__ double s_sum[kThreads][8];
@@ -335,7 +373,6 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
   __shared__ uint64_t bar;
   const int bh = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
-  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
   if (threadIdx.x < D) {
     const int c = threadIdx.x;
     if (IS_K) {
@@ -349,34 +386,7 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
     }
   }
   if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh)) return;
-  if (!IS_K && SHIFT) {
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
-      double cs[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) cs[e] = 0.0;
-#pragma unroll
-      for (int p = nb * PPB; p < (nb + 1) * PPB; ++p) {
-        float x[8];
-        lds8(sX + (rg + p * RG) * D + ch * 8, x);  // rows past N are zero
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cs[e] += (double)x[e];
-      }
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
-      __syncthreads();
-      if (threadIdx.x < D) {
-        const int c = threadIdx.x;
-        double s = 0.0;
-        for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
-        const float mu = vb > 0 ? __double2float_rn(__ddiv_rn(s, (double)vb)) : 0.0f;
-        s_shift[nb][c] = mu;
-        if (vb > 0) a.qbar[((int64_t)bh * a.Tm + tile * NB + nb) * D + c] = mu;
-      }
-    }
-  }
+  if (!IS_K && SHIFT) block_means<T, D, BQ>(sX, s_sum, s_shift, bh, tile, a);
   __syncthreads();
   qk_encode<T, D, BQ, IS_K, SHIFT>(sX, s_shift, s_red, s_bmax, bh, tile, a);
 }

@@ -91,74 +91,124 @@ __global__ void __launch_bounds__(kThreads) k_quant_nvfp4_kernel(QuantArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Q: optional per-BQ-block mean (smooth Q), NVFP4 along d.  One 128-row tile
-// per CTA (128 / BQ mean blocks).  grid (Np/128, B*Hq), 256 threads.
+// NVFP4 codes of one 128-row tile in shared memory (rows past N are zero):
+// x - shift[row block] for the valid rows (shift == nullptr: no shift), one
+// E4M3 scale per 16 channels, codes to x4 (this tile's rows), scales to the
+// tile's 1 KB block sf.  Every thread of the CTA calls it.
 template <typename T, int BQ>
-__global__ void __launch_bounds__(kThreads) q_quant_nvfp4_kernel(QuantArgs a) {
-  constexpr int D = kF4D, CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NB = kTile / BQ, PPB = BQ / RG;
-  __shared__ double s_sum[kThreads][8];
-  __shared__ float s_mean[NB][D];
-  __shared__ __align__(16) uint8_t s_sf[1024];
-  const int bh = blockIdx.y, tile = blockIdx.x;
-  const int64_t r0 = (int64_t)tile * kTile;
-  const int valid = rows_valid(a.N, r0, kTile);
+__device__ __forceinline__ void nvfp4_encode_tile(const T* sX, const float (*shift)[kF4D], uint8_t* s_sf, int valid,
+                                                  uint8_t* x4, uint8_t* sf) {
+  constexpr int D = kF4D, CH = D / 8, RG = kThreads / CH, NP = kTile / RG, PPB = BQ / RG;
   const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
-  const T* Q = reinterpret_cast<const T*>(a.q) + (int64_t)bh * a.N * D;
-  float x[NP][8];
-#pragma unroll
+#pragma unroll 4
   for (int p = 0; p < NP; ++p) {
     const int r = rg + p * RG;
-    if (r < valid) {
-      load8<T>(Q + (r0 + r) * D + ch * 8, x[p]);
-    } else {
+    float x[8];
+    lds8(sX + r * D + ch * 8, x);
+    if (shift != nullptr && r < valid) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[p][e] = 0.0f;
+      for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], shift[p / PPB][ch * 8 + e]);
     }
-  }
-  if (a.smooth_q) {
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int vb = rows_valid(a.N, r0 + nb * BQ, BQ);
-      double cs[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) cs[e] = 0.0;
-#pragma unroll
-      for (int p = nb * PPB; p < (nb + 1) * PPB; ++p)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cs[e] += (double)x[p][e];  // invalid rows hold 0
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s_sum[threadIdx.x][e] = cs[e];
-      __syncthreads();
-      if (threadIdx.x < D) {
-        const int c = threadIdx.x;
-        double s = 0.0;
-        for (int g = 0; g < RG; ++g) s += s_sum[g * CH + c / 8][c % 8];
-        const float mu = vb > 0 ? __double2float_rn(__ddiv_rn(s, (double)vb)) : 0.0f;
-        s_mean[nb][c] = mu;
-        const int blk = tile * NB + nb;
-        if (vb > 0) a.qbar[((int64_t)bh * a.Tm + blk) * D + c] = mu;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int p = 0; p < NP; ++p)
-      if (rg + p * RG < valid)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[p][e] = __fsub_rn(x[p][e], s_mean[p / PPB][ch * 8 + e]);
-  }
-  uint8_t* q4 = a.q4 + ((int64_t)bh * a.Np + r0) * (D / 2);
-#pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
     uint32_t sc;
-    const uint32_t codes = encode_pair(x[p], &sc);
-    *reinterpret_cast<uint32_t*>(q4 + r * (D / 2) + ch * 4) = codes;
+    const uint32_t codes = encode_pair(x, &sc);
+    *reinterpret_cast<uint32_t*>(x4 + r * (D / 2) + ch * 4) = codes;
     if ((ch & 1) == 0) s_sf[sf_byte(r, ch >> 1)] = (uint8_t)sc;
   }
   __syncthreads();
-  reinterpret_cast<uint32_t*>(a.sfq + ((int64_t)bh * (a.Np / kTile) + tile) * 1024)[threadIdx.x] =
-      reinterpret_cast<const uint32_t*>(s_sf)[threadIdx.x];
+  reinterpret_cast<uint32_t*>(sf)[threadIdx.x] = reinterpret_cast<const uint32_t*>(s_sf)[threadIdx.x];
+}
+
+// Q: optional per-BQ-block mean (smooth Q), NVFP4 along d.  One 128-row tile
+// per CTA, staged in shared memory by one TMA load (3D map, rows past N read
+// as zeros).  grid (Np/128, B*Hq), 256 threads, dynamic smem 128 x 128
+// elements + 128.
+template <typename T, int BQ, bool SHIFT>
+__global__ void __launch_bounds__(kThreads) q_quant_nvfp4_kernel(const __grid_constant__ CUtensorMap tmQ, QuantArgs a) {
+  constexpr int D = kF4D, NB = kTile / BQ;
+  extern __shared__ uint8_t q4_smem_raw[];
+  T* sX = reinterpret_cast<T*>(align128(q4_smem_raw));
+  __shared__ double s_sum[SHIFT ? kThreads : 1][8];
+  __shared__ float s_mean[NB][D];
+  __shared__ __align__(16) uint8_t s_sf[1024];
+  __shared__ uint64_t bar;
+  const int bh = blockIdx.y, tile = blockIdx.x;
+  const int64_t r0 = (int64_t)tile * kTile;
+  if (!load_tile<T, D>(sX, &tmQ, &bar, (int)r0, bh)) return;
+  if (SHIFT) block_means<T, D, BQ>(sX, s_sum, s_mean, bh, tile, a);
+  __syncthreads();
+  nvfp4_encode_tile<T, BQ>(sX, SHIFT ? s_mean : nullptr, s_sf, rows_valid(a.N, r0, kTile),
+                           a.q4 + ((int64_t)bh * a.Np + r0) * (D / 2),
+                           a.sfq + ((int64_t)bh * (a.Np / kTile) + tile) * 1024);
+}
+
+// ---------------------------------------------------------------------------
+// One-read K: each CTA loads one 128-token tile of K once and keeps it in
+// shared memory while its head's column sums complete (the scheme of the
+// INT8 path's one-read K/V kernel: tickets in CTA start order, fp64 atomics,
+// a publish counter per head, bounded waits), then encodes gamma(K) = K - km.
+// Ticket t: head t / tiles, tile t % tiles.  grid (tiles B Hkv), 256 threads,
+// dynamic smem 128 x 128 elements + 128.
+template <typename T, bool SMOOTH_K>
+__global__ void __launch_bounds__(kThreads) k_fused_nvfp4_kernel(const __grid_constant__ CUtensorMap tmK, QuantArgs a) {
+  constexpr int D = kF4D, CH = D / 8, RG = kThreads / CH, NP = kTile / RG, NW = kThreads / 32;
+  extern __shared__ uint8_t k4_smem_raw[];
+  T* sX = reinterpret_cast<T*>(align128(k4_smem_raw));
+  __shared__ double s_pk[SMOOTH_K ? NW * D : 1];
+  __shared__ float s_km[1][D];
+  __shared__ __align__(16) uint8_t s_sf[1024];
+  __shared__ uint64_t bar;
+  __shared__ int s_item, s_ok;
+  const int tiles = (int)(a.Np / kTile);
+  if (threadIdx.x == 0) s_item = atomicAdd(a.kv_sync, 1);
+  __syncthreads();
+  const int bg = s_item / tiles, tile = s_item % tiles;
+  if (!load_tile<T, D>(sX, &tmK, &bar, tile * kTile, bg)) return;
+  if constexpr (SMOOTH_K) {
+    const int ch = threadIdx.x % CH, rg = threadIdx.x / CH, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    double cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      float x[8];
+      lds8(sX + (rg + p * RG) * D + ch * 8, x);  // rows past N are zero
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] += (double)x[e];
+    }
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], o);
+    if (lane < CH)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_pk[warp * D + ch * 8 + e] = cs[e];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      double sum = 0.0;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) sum += s_pk[w * D + threadIdx.x];
+      atomicAdd(a.ksum + (int64_t)bg * D + threadIdx.x, sum);
+      __threadfence();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      atomicAdd(a.kv_sync + 1 + bg, 1);
+      s_ok = wait_count(a.kv_sync + 1 + bg, tiles) ? 1 : 0;  // every tile of the head added its sums
+    }
+    __syncthreads();
+    if (!s_ok) return;  // timeout recorded; this tile's codes are not written
+    if (threadIdx.x < D) {
+      const float km = __double2float_rn(__ddiv_rn(__ldcg(a.ksum + (int64_t)bg * D + threadIdx.x), (double)a.N));
+      s_km[0][threadIdx.x] = km;
+      if (tile == 0) a.km[(int64_t)bg * D + threadIdx.x] = km;
+    }
+  } else {
+    if (threadIdx.x < D && tile == 0) a.km[(int64_t)bg * D + threadIdx.x] = 0.0f;
+  }
+  __syncthreads();
+  nvfp4_encode_tile<T, kTile>(sX, SMOOTH_K ? s_km : nullptr, s_sf, rows_valid(a.N, (int64_t)tile * kTile, kTile),
+                              a.k4 + ((int64_t)bg * a.Np + (int64_t)tile * kTile) * (D / 2),
+                              a.sfk + ((int64_t)bg * (a.Np / kTile) + tile) * 1024);
 }
 
 // ---------------------------------------------------------------------------
@@ -223,24 +273,59 @@ __global__ void __launch_bounds__(kThreads) v_quant_nvfp4_kernel(QuantArgs a) {
       reinterpret_cast<const uint32_t*>(s_sf)[threadIdx.x];
 }
 
+using KNvfp4Fn = void (*)(CUtensorMap, QuantArgs);
+
+// The one-read K kernel, or nullptr if one head's `tiles` CTAs might not fit
+// in half of the CTAs resident at once (then statistics + K kernels run).
 template <typename T>
-cudaError_t launch_quant_nvfp4_t(const QuantArgs& a, cudaStream_t st) {
+KNvfp4Fn k_fused_nvfp4_for(const QuantArgs& a, int tiles, int smem) {
+  KNvfp4Fn kf = a.smooth_k ? k_fused_nvfp4_kernel<T, true> : k_fused_nvfp4_kernel<T, false>;
+  if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return nullptr;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kf, kThreads, smem) != cudaSuccess)
+    return nullptr;
+  return (int64_t)tiles * 2 <= (int64_t)sms * per_sm ? kf : nullptr;
+}
+
+template <typename T>
+int quant_nvfp4_kernel_count_t(const QuantArgs& a, bool allow_one_read) {
+  const int tiles = (int)(a.Np / kTile);
+  const bool one_read = allow_one_read && k_fused_nvfp4_for<T>(a, tiles, kTile * kF4D * (int)sizeof(T) + 128);
+  return (one_read ? 1 : 2) + 2 + (a.smooth_q ? 1 : 0);
+}
+
+template <typename T>
+cudaError_t launch_quant_nvfp4_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t st) {
   cudaError_t e;
   const int BHkv = a.B * a.Hkv, BHq = a.B * a.Hq;
   const int tiles = (int)(a.Np / kTile);
+  const int smem = kTile * kF4D * (int)sizeof(T) + 128;
   QuantArgs s = a;
   s.vamax = nullptr;  // no per-channel V statistics on this path
-  if (a.smooth_k) {
-    e = cudaMemsetAsync(a.ksum, 0, sizeof(double) * (size_t)BHkv * kF4D, st);
+  auto kf = a.kv_sync ? k_fused_nvfp4_for<T>(a, tiles, smem) : nullptr;
+  if (kf) {
+    // ksum and kv_sync are consecutive in the workspace: one memset
+    e = cudaMemsetAsync(a.ksum, 0, a.kv_zero_bytes, st);
     if (e != cudaSuccess) return e;
+    kf<<<dim3(tiles * BHkv), kThreads, smem, st>>>(m.k, s);
+  } else {
+    if (a.smooth_k) {
+      e = cudaMemsetAsync(a.ksum, 0, sizeof(double) * (size_t)BHkv * kF4D, st);
+      if (e != cudaSuccess) return e;
+    }
+    kv_stats_kernel<T, kF4D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(s);
+    k_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, 0, st>>>(s);
   }
-  kv_stats_kernel<T, kF4D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(s);
-  k_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, 0, st>>>(s);
   v_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, 0, st>>>(s);
-  if (a.bq == 64)
-    q_quant_nvfp4_kernel<T, 64><<<dim3(tiles, BHq), kThreads, 0, st>>>(s);
-  else
-    q_quant_nvfp4_kernel<T, 128><<<dim3(tiles, BHq), kThreads, 0, st>>>(s);
+  {
+    auto qq = a.bq == 64 ? (a.smooth_q ? q_quant_nvfp4_kernel<T, 64, true> : q_quant_nvfp4_kernel<T, 64, false>)
+                         : (a.smooth_q ? q_quant_nvfp4_kernel<T, 128, true> : q_quant_nvfp4_kernel<T, 128, false>);
+    e = cudaFuncSetAttribute(qq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    qq<<<dim3(tiles, BHq), kThreads, smem, st>>>(m.q, s);
+  }
   if (a.smooth_q) {
     e = launch_delta_s<T, kF4D>(s, st);
     if (e != cudaSuccess) return e;
@@ -250,9 +335,14 @@ cudaError_t launch_quant_nvfp4_t(const QuantArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_quant_nvfp4(const QuantArgs& a, int is_fp16, cudaStream_t st) {
+cudaError_t launch_quant_nvfp4(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st) {
   if (a.D != kF4D) return cudaErrorInvalidValue;
-  return is_fp16 ? launch_quant_nvfp4_t<__half>(a, st) : launch_quant_nvfp4_t<__nv_bfloat16>(a, st);
+  return is_fp16 ? launch_quant_nvfp4_t<__half>(a, m, st) : launch_quant_nvfp4_t<__nv_bfloat16>(a, m, st);
+}
+
+int quant_nvfp4_kernel_count(const QuantArgs& a, int is_fp16, bool allow_one_read) {
+  return is_fp16 ? quant_nvfp4_kernel_count_t<__half>(a, allow_one_read)
+                 : quant_nvfp4_kernel_count_t<__nv_bfloat16>(a, allow_one_read);
 }
 
 }  // namespace sage

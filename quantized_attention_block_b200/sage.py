@@ -28,7 +28,7 @@ EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized",
             "sage_status_string", "sage_attn_fwd_noalloc", "sage_debug_f8_accum_probe",
             "sage_nvfp4_workspace_bytes", "sage_quant_nvfp4", "sage_attn_fwd_nvfp4_quantized",
             "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4", "sage_debug_exp2_poly",
-            "sage_debug_kv_quant_two_pass", "sage_quant_kernel_count")
+            "sage_debug_kv_quant_two_pass", "sage_quant_kernel_count", "sage_quant_nvfp4_kernel_count")
 
 
 class SageError(RuntimeError):
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.sage_debug_kv_quant_two_pass.argtypes, L.sage_debug_kv_quant_two_pass.restype = [i32], ctypes.c_int
         L.sage_quant_kernel_count.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         L.sage_quant_kernel_count.restype = ctypes.c_int
+        L.sage_quant_nvfp4_kernel_count.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
+        L.sage_quant_nvfp4_kernel_count.restype = ctypes.c_int
         for n in ("sage_quant_qkv", "sage_attn_fwd_quantized", "sage_attn_fwd", "sage_debug_qk_int32",
                   "sage_last_device_error", "sage_debug_bounded_wait", "sage_quant_nvfp4",
                   "sage_attn_fwd_nvfp4_quantized", "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4"):
@@ -279,6 +281,13 @@ def sage_quant_kernel_count(p: SageParams) -> int:
     """Kernels sage_quant_qkv enqueues for p on the current device (memsets not counted)."""
     n = ctypes.c_int32(0)
     _check(lib().sage_quant_kernel_count(ctypes.byref(p), ctypes.byref(n)), "sage_quant_kernel_count")
+    return int(n.value)
+
+
+def sage_quant_nvfp4_kernel_count(p: SageParams) -> int:
+    """Kernels sage_quant_nvfp4 enqueues for p on the current device (memsets not counted)."""
+    n = ctypes.c_int32(0)
+    _check(lib().sage_quant_nvfp4_kernel_count(ctypes.byref(p), ctypes.byref(n)), "sage_quant_nvfp4_kernel_count")
     return int(n.value)
 
 

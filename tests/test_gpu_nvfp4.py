@@ -44,6 +44,41 @@ def test_nvfp4_quant_bit_exact(name):
     assert not bad, bad
 
 
+@pytest.mark.parametrize("name", list(ALL))
+def test_nvfp4_one_read_k_equals_two_pass(name):
+    """The one-read K kernel (each tile waits in shared memory for its head's
+    column sums) and the statistics-pass path write the same bytes."""
+    w = ALL[name]
+    q, k, v = W.make_qkv(w)
+    p, ws1, view1, _ = gpu_quant_nvfp4(w, q, k, v)
+    assert sage.sage_last_device_error() == 0
+    sage.sage_debug_kv_quant_two_pass(True)
+    try:
+        _, ws2, view2, _ = gpu_quant_nvfp4(w, q, k, v)
+    finally:
+        sage.sage_debug_kv_quant_two_pass(False)
+    assert sage.sage_last_device_error() == 0
+    t1, t2 = sage.nvfp4_view_tensors(view1, p, ws1), sage.nvfp4_view_tensors(view2, p, ws2)
+    assert t1.keys() == t2.keys()
+    for key in t1:
+        a = t1[key].contiguous().cpu().numpy()
+        b = t2[key].contiguous().cpu().numpy()
+        np.testing.assert_array_equal(a.reshape(-1).view(np.uint8), b.reshape(-1).view(np.uint8), err_msg=key)
+
+
+def test_nvfp4_quant_kernel_count_follows_the_path():
+    w = NV
+    p = sage.SageParams(w.B, w.Hq, w.Hkv, w.N, w.d, 0, int(w.causal), float(w.sm_scale or 0.0),
+                        int(w.smooth_k), int(w.smooth_q), w.bq, w.bk, 0)
+    extra = 1 if w.smooth_q else 0
+    assert sage.sage_quant_nvfp4_kernel_count(p) == 3 + extra
+    sage.sage_debug_kv_quant_two_pass(True)
+    try:
+        assert sage.sage_quant_nvfp4_kernel_count(p) == 4 + extra
+    finally:
+        sage.sage_debug_kv_quant_two_pass(False)
+
+
 @pytest.mark.parametrize("name", ["nvfp4_N600", "N384_gqa_no_smooth_k"])
 def test_nvfp4_qk_tile_matches_exact_dot_products(name):
     """The block-scaled MMA tile against the exact sums of the exact products
