@@ -701,88 +701,100 @@ __global__ void __launch_bounds__(kThreads, 2) delta_s_tc_kernel(QuantArgs a) {
   float* out = a.dS + (int64_t)bh * a.Tm * a.Np + r0;
   const int quarter = warp & 3, half = warp >> 2;
   const int cl = (threadIdx.x % G8) * 8;  // this thread's channels within a pass (every step)
+  // Passes (chunk of NBK Q blocks, 64 channels) run in order; the global loads
+  // of pass p + 1 are issued as soon as pass p's operands are in shared memory,
+  // so they are in flight during pass p's MMAs and stores (the registers that
+  // hold them are free by then).
+  constexpr int NPC = D / CP;  // passes per chunk
+  constexpr int ITA = kTile * G8 / kThreads, ITB = (NBK * G8 + kThreads - 1) / kThreads;
+  const int n_pass = ((a.Tm + NBK - 1) / NBK) * NPC;
+  uint4 ka[ITA];
+  float4 qv[ITB][2];
+  // A = gamma(K)[:, c0 .. c0 + 64) (rows past N zero; with a single pass per
+  // chunk (d = 64) A stays from the first chunk), B = qbar[i0 .., c0 ..) (rows
+  // past Tm zero)
+  auto load_pass = [&](int pass) {
+    const int pi0 = (pass / NPC) * NBK, pc0 = (pass % NPC) * CP;
+    const int pnb = min(NBK, a.Tm - pi0);
+    const bool load_a = D > CP || pi0 == 0;
+#pragma unroll
+    for (int it = 0; it < ITA; ++it) {
+      const int r = (threadIdx.x + it * kThreads) / G8;
+      ka[it] = (load_a && r < valid) ? __ldg(reinterpret_cast<const uint4*>(K + (int64_t)r * D + pc0 + cl))
+                                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int it = 0; it < ITB; ++it) {
+      const int r = (threadIdx.x + it * kThreads) / G8;
+      const float* src = qb + (int64_t)(pi0 + r) * D + pc0 + cl;
+      qv[it][0] = r < pnb ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      qv[it][1] = r < pnb ? __ldg(reinterpret_cast<const float4*>(src + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
   bool ok = true;
   uint32_t phase = 0;
-  for (int i0 = 0; i0 < a.Tm && ok; i0 += NBK) {
+  load_pass(0);
+  for (int pass = 0; pass < n_pass && ok; ++pass, phase ^= 1u) {
+    const int i0 = (pass / NPC) * NBK, c0 = (pass % NPC) * CP;
     const int nb = min(NBK, a.Tm - i0);
     const int nbp = (nb + 15) & ~15;  // MMA N: a multiple of 16
     const uint32_t idesc = make_idesc(/*F32*/ 1, /*TF32*/ 2, /*TF32*/ 2, kTile, nbp);
-    for (int c0 = 0; c0 < D && ok; c0 += CP, phase ^= 1u) {
-      // A = gamma(K)[:, c0 .. c0 + 64) (rows past N zero), B = qbar[i0 .., c0 ..)
-      // (rows past Tm zero); every load of the thread is issued before use.
-      // With a single pass (d = 64) A stays from the first chunk.
-      const bool load_a = D > CP || i0 == 0;
-      constexpr int ITA = kTile * G8 / kThreads, ITB = (NBK * G8 + kThreads - 1) / kThreads;
-      uint4 ka[ITA];
-      float4 qv[ITB][2];
+    const bool load_a = D > CP || i0 == 0;
+    float kmc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) kmc[e] = km[c0 + cl + e];
+    // the previous pass's MMAs have read the operands (waited on below)
+    if (load_a) {
 #pragma unroll
       for (int it = 0; it < ITA; ++it) {
         const int r = (threadIdx.x + it * kThreads) / G8;
-        ka[it] = (load_a && r < valid) ? __ldg(reinterpret_cast<const uint4*>(K + (int64_t)r * D + c0 + cl))
-                                       : make_uint4(0u, 0u, 0u, 0u);
+        float x[8];
+        lds8(reinterpret_cast<const T*>(&ka[it]), x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = r < valid ? __fsub_rn(x[e], kmc[e]) : 0.0f;
+        store_split8(sAh, sAl, r, cl, kTile, x);
       }
-#pragma unroll
-      for (int it = 0; it < ITB; ++it) {
-        const int r = (threadIdx.x + it * kThreads) / G8;
-        const float* src = qb + (int64_t)(i0 + r) * D + c0 + cl;
-        qv[it][0] = r < nb ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        qv[it][1] = r < nb ? __ldg(reinterpret_cast<const float4*>(src + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      float kmc[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) kmc[e] = km[c0 + cl + e];
-      // the previous pass's MMAs have read the operands (waited on below)
-      if (load_a) {
-#pragma unroll
-        for (int it = 0; it < ITA; ++it) {
-          const int r = (threadIdx.x + it * kThreads) / G8;
-          float x[8];
-          lds8(reinterpret_cast<const T*>(&ka[it]), x);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = r < valid ? __fsub_rn(x[e], kmc[e]) : 0.0f;
-          store_split8(sAh, sAl, r, cl, kTile, x);
-        }
-      }
-#pragma unroll
-      for (int it = 0; it < ITB; ++it) {
-        const int r = (threadIdx.x + it * kThreads) / G8;
-        if (r < nbp) {
-          const float x[8] = {qv[it][0].x, qv[it][0].y, qv[it][0].z, qv[it][0].w,
-                              qv[it][1].x, qv[it][1].y, qv[it][1].z, qv[it][1].w};
-          store_split8(sBh, sBl, r, cl, NBK, x);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        tc_fence_after();
-        const uint32_t aH = smem_u32(sAh), aL = smem_u32(sAl), bH = smem_u32(sBh), bL = smem_u32(sBl);
-        // K step kk: 8 channels = 32 bytes inside 32-channel column block kk / 4
-#pragma unroll
-        for (int kk = 0; kk < CP / 8; ++kk) {
-          const uint32_t oa = (kk >> 2) * kTile * 128 + (kk & 3) * 32, ob = (kk >> 2) * NBK * 128 + (kk & 3) * 32;
-          mma_tf32(tmem, make_sdesc(aH + oa, 1024, kSwizzle128B), make_sdesc(bL + ob, 1024, kSwizzle128B), idesc,
-                   (c0 > 0 || kk > 0) ? 1u : 0u);
-          mma_tf32(tmem, make_sdesc(aL + oa, 1024, kSwizzle128B), make_sdesc(bH + ob, 1024, kSwizzle128B), idesc,
-                   1u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < CP / 8; ++kk) {
-          const uint32_t oa = (kk >> 2) * kTile * 128 + (kk & 3) * 32, ob = (kk >> 2) * NBK * 128 + (kk & 3) * 32;
-          mma_tf32(tmem, make_sdesc(aH + oa, 1024, kSwizzle128B), make_sdesc(bH + ob, 1024, kSwizzle128B), idesc,
-                   1u);
-        }
-        mma_commit(&mma_bar);
-      }
-      __syncwarp();
-      ok = mbar_wait_warp(&mma_bar, phase);
-      tc_fence_after();
-      ok = __syncthreads_and(ok);
     }
-    if (ok) {
-      // lanes 32 quarter ..: keys; the two halves of the CTA take alternate
-      // 16-block groups
+#pragma unroll
+    for (int it = 0; it < ITB; ++it) {
+      const int r = (threadIdx.x + it * kThreads) / G8;
+      if (r < nbp) {
+        const float x[8] = {qv[it][0].x, qv[it][0].y, qv[it][0].z, qv[it][0].w,
+                            qv[it][1].x, qv[it][1].y, qv[it][1].z, qv[it][1].w};
+        store_split8(sBh, sBl, r, cl, NBK, x);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      const uint32_t aH = smem_u32(sAh), aL = smem_u32(sAl), bH = smem_u32(sBh), bL = smem_u32(sBl);
+      // K step kk: 8 channels = 32 bytes inside 32-channel column block kk / 4
+#pragma unroll
+      for (int kk = 0; kk < CP / 8; ++kk) {
+        const uint32_t oa = (kk >> 2) * kTile * 128 + (kk & 3) * 32, ob = (kk >> 2) * NBK * 128 + (kk & 3) * 32;
+        mma_tf32(tmem, make_sdesc(aH + oa, 1024, kSwizzle128B), make_sdesc(bL + ob, 1024, kSwizzle128B), idesc,
+                 (c0 > 0 || kk > 0) ? 1u : 0u);
+        mma_tf32(tmem, make_sdesc(aL + oa, 1024, kSwizzle128B), make_sdesc(bH + ob, 1024, kSwizzle128B), idesc,
+                 1u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < CP / 8; ++kk) {
+        const uint32_t oa = (kk >> 2) * kTile * 128 + (kk & 3) * 32, ob = (kk >> 2) * NBK * 128 + (kk & 3) * 32;
+        mma_tf32(tmem, make_sdesc(aH + oa, 1024, kSwizzle128B), make_sdesc(bH + ob, 1024, kSwizzle128B), idesc,
+                 1u);
+      }
+      mma_commit(&mma_bar);
+    }
+    if (pass + 1 < n_pass) load_pass(pass + 1);
+    __syncwarp();
+    ok = mbar_wait_warp(&mma_bar, phase);
+    tc_fence_after();
+    ok = __syncthreads_and(ok);
+    if (ok && c0 + CP == D) {
+      // the chunk's accumulator is complete.  Lanes 32 quarter ..: keys; the two
+      // halves of the CTA take alternate 16-block groups
       const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
       const int key = quarter * 32 + lane;
       for (int g = half; g < nbp / 16; g += 2) {
@@ -795,11 +807,11 @@ __global__ void __launch_bounds__(kThreads, 2) delta_s_tc_kernel(QuantArgs a) {
           if (i < a.Tm) out[(int64_t)i * a.Np + key] = __uint_as_float(v[e]);
         }
       }
+      // every warp has read the accumulator before the next chunk's MMAs
+      tc_fence_before();
+      ok = __syncthreads_and(ok);
+      tc_fence_after();
     }
-    // every warp has read the accumulator before the next chunk's MMAs
-    tc_fence_before();
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
   }
   tc_fence_before();
   __syncthreads();
