@@ -65,7 +65,8 @@ typedef struct {
     float   sm_scale;          /* softmax scale; <= 0 selects 1/sqrt(d) */
     int32_t smooth_k;          /* 1: subtract the per-(b, kv-head, channel) token mean of K */
     int32_t smooth_q;          /* 1: subtract each Q block's mean and add delta_S back */
-    int32_t bq;                /* Q quantisation block in rows: 64 or 128 */
+    int32_t bq;                /* Q quantisation block in rows: 32, 64 or 128 (32: one
+                                  scale per 32-row TMEM lane group; INT8/FP8 path only) */
     int32_t bk;                /* K quantisation block in rows: 64 or 128 */
     int32_t pv_accum;          /* FP32 accumulation of P~V across key tiles:
                                   SAGE_PV_TWO_LEVEL (0): each tile's P^V lands in a

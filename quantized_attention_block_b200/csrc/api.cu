@@ -39,7 +39,7 @@ sage_status check_params(const sage_params* p, Dims* d) {
   if (p->Hq % p->Hkv != 0) return SAGE_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SAGE_ERR_UNSUPPORTED_HEADDIM;
   if (p->dtype != SAGE_BF16 && p->dtype != SAGE_FP16) return SAGE_ERR_UNSUPPORTED_DTYPE;
-  if ((p->bq != 64 && p->bq != 128) || (p->bk != 64 && p->bk != 128)) return SAGE_ERR_INVALID_ARG;
+  if ((p->bq != 32 && p->bq != 64 && p->bq != 128) || (p->bk != 64 && p->bk != 128)) return SAGE_ERR_INVALID_ARG;
   if ((p->causal != 0 && p->causal != 1) || (p->smooth_k != 0 && p->smooth_k != 1) ||
       (p->smooth_q != 0 && p->smooth_q != 1))
     return SAGE_ERR_INVALID_ARG;
@@ -234,6 +234,7 @@ LayoutF4 make_layout_f4(const sage_params* p, const Dims& d) {
 sage_status check_params_f4(const sage_params* p, Dims* d) {
   const sage_status s = check_params(p, d);
   if (s != SAGE_OK) return s;
+  if (p->bq == 32) return SAGE_ERR_INVALID_ARG;  // the NVFP4 smooth-Q block is 64 or 128 rows
   return d->D == 128 ? SAGE_OK : SAGE_ERR_UNSUPPORTED_HEADDIM;
 }
 

@@ -80,7 +80,7 @@ struct Smem {
   static constexpr uint32_t oK = oQ + 2 * kQ;            // kStages
   static constexpr uint32_t oV = oK + kStages * kK;      // kStages
   static constexpr uint32_t oP = oV + kStages * kV;      // [tile][2 buffers]
-  static constexpr uint32_t kDS = 2 * 2 * 128 * 4;      // delta_S rows of one key tile
+  static constexpr uint32_t kDS = 2 * 4 * 128 * 4;      // delta_S rows of one key tile: [tile][Q block (<= 4)][128]
   static constexpr uint32_t oDS = oP + 4 * kP;           // kStages
   static constexpr uint32_t oAlpha = oDS + kStages * kDS;  // float[tile][buffer][128]
   static constexpr uint32_t oL = oAlpha + 4 * 128 * 4;   // float[2][128]
@@ -88,6 +88,7 @@ struct Smem {
   static constexpr uint32_t kNumBars = 1 + 3 * kStages + 2 + 4 + 4 + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = oTmem + 16 + 1024;  // + alignment slack
+  static_assert(kBytes <= 227 * 1024, "attention tile buffers exceed the shared memory of one CTA");
 };
 
 template <typename TO>
@@ -227,7 +228,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
       const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np);
       const int vrow = (b * a.Hkv + g) * D;
-      const int ds_rows = kTile / a.bq;  // Q blocks per tile (1 or 2)
+      const int ds_rows = kTile / a.bq;  // Q blocks per tile (1, 2 or 4)
       const uint32_t ds_bytes = (uint32_t)((nTi[0] > 0) + (nTi[1] > 0)) * ds_rows * 512;
       mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
       for (int i = 0; i < 2; ++i)
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             for (int hb = 0; hb < ds_rows; ++hb)
               if (nTi[i] > 0) {
                 const int blk = min((2 * pr + i) * ds_rows + hb, a.Tm - 1);
-                bulk_load_1d(smem + L::oDS + s * L::kDS + (i * 2 + hb) * 512,
+                bulk_load_1d(smem + L::oDS + s * L::kDS + (i * 4 + hb) * 512,
                              a.dS + ((int64_t)(b * a.Hq + h) * a.Tm + blk) * a.Np + (int64_t)j * kTile, 512,
                              &bar.k_full[s]);
               }
@@ -353,7 +354,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const int qblk = min((int)(qrow / a.bq), a.Tm - 1);
     const float row_scale = a.s_q[(int64_t)(b * a.Hq + h) * a.Tm + qblk] * a.scale_log2;
     const float* sk = a.s_k + (int64_t)(b * a.Hkv + g) * a.Tn;
-    const int ds_half = (a.bq == 64 && row >= 64) ? 1 : 0;  // warp-uniform
+    // this row's Q block within the tile (warp-uniform: bq >= 32); a shift, not a
+    // division by the runtime bq (which the compiler would redo in the tile loop)
+    const int ds_blk = row >> (a.bq == 32 ? 5 : (a.bq == 64 ? 6 : 7));
     float sk_lo = __ldg(sk + 0), sk_hi = __ldg(sk + min(64 / a.bk, a.Tn - 1));
     const float sl2 = a.scale_log2;
     const float2 neg_magic = make_float2(-kMagic, -kMagic);
@@ -375,7 +378,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       // next tile's key-block scales (their load latency hides behind this tile)
       sk_lo = __ldg(sk + min((col0 + kTile) / a.bk, a.Tn - 1));
       sk_hi = __ldg(sk + min((col0 + kTile + 64) / a.bk, a.Tn - 1));
-      const float* dsr = sDS + (j % kStages) * (L::kDS / 4) + (ti * 2 + ds_half) * 128;
+      const float* dsr = sDS + (j % kStages) * (L::kDS / 4) + (ti * 4 + ds_blk) * 128;
       if (HAS_DS && !(ok = mbar_wait_warp(&bar.k_full[j % kStages], (j / kStages) & 1))) break;
       tmem_ld_wait();
       if (!TWO_LEVEL) {

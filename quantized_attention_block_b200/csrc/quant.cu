@@ -884,8 +884,9 @@ cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t 
     v_quant_kernel<T, D><<<dim3(tiles, BHkv), kThreads, smem, st>>>(m.v, m.vt, a);
   }
   {
-    auto qq = a.bq == 64 ? (a.smooth_q ? qk_quant_kernel<T, D, 64, false, true> : qk_quant_kernel<T, D, 64, false, false>)
-                         : (a.smooth_q ? qk_quant_kernel<T, D, 128, false, true> : qk_quant_kernel<T, D, 128, false, false>);
+    auto qq = a.bq == 32   ? (a.smooth_q ? qk_quant_kernel<T, D, 32, false, true> : qk_quant_kernel<T, D, 32, false, false>)
+              : a.bq == 64 ? (a.smooth_q ? qk_quant_kernel<T, D, 64, false, true> : qk_quant_kernel<T, D, 64, false, false>)
+                           : (a.smooth_q ? qk_quant_kernel<T, D, 128, false, true> : qk_quant_kernel<T, D, 128, false, false>);
     e = cudaFuncSetAttribute(qq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_qk);
     if (e != cudaSuccess) return e;
     qq<<<dim3(tiles, BHq), kThreads, smem_qk, st>>>(m.q, a);

@@ -31,6 +31,11 @@ EDGE = {
     "N257_smoothq_causal_d128": W.get("gqa").with_(name="N257_sq", B=1, Hq=2, Hkv=2, N=257, smooth_q=True,
                                                    qk_shared_bias_std=2.0, k_bias_std=0.0),
     "N513_bq64_bk64_d64": W.get("video").with_(name="N513", B=1, Hq=1, Hkv=1, N=513, bq=64),
+    # one Q scale per 32-row TMEM lane group
+    "N300_bq32_causal": W.get("prefill").with_(name="N300_bq32", B=1, Hq=2, Hkv=2, N=300, bq=32),
+    "N385_bq32_smoothq_d64": W.get("video").with_(name="N385_bq32", B=1, Hq=2, Hkv=2, N=385, bq=32),
+    "N260_bq32_smoothq_gqa_causal": W.get("gqa").with_(name="N260_bq32_sq", B=1, Hq=4, Hkv=2, N=260, bq=32,
+                                                        smooth_q=True, qk_shared_bias_std=0.0, k_bias_std=3.0),
 }
 
 
