@@ -54,7 +54,7 @@ def lib():
         L.or_delta_s.argtypes = [P, i64, P, P, i64, i32, P]
         L.or_quant_nvfp4_rows.argtypes = [P, i64, i32, i32, P, i32, P, P]
         L.or_quant_nvfp4_cols.argtypes = [P, i64, i32, P, P]
-        L.or_attn_core.argtypes = [P, P, P, P, P, P, i32, P, i64, i32, i32, i32, f64, i32, i32, i64, i64, P]
+        L.or_attn_core.argtypes = [P, P, P, P, P, P, i32, P, i64, i32, i32, i32, f64, i32, i32, i64, i64, P, P]
         L.or_attn_naive_f64.argtypes = [P, P, P, i64, i32, i32, f64, i64, i64, P]
         for name in ("or_mean_rows", "or_block_means", "or_quant_int8", "or_quant_fp8_per_channel",
                      "or_delta_s", "or_quant_nvfp4_rows", "or_quant_nvfp4_cols", "or_attn_core",
@@ -243,18 +243,22 @@ def quantize_sage(q, k, v, *, bq: int, bk: int, smooth_k: bool = True, smooth_q:
 
 # ---------------------------------------------------------------- attention
 def _attn_core(Qv, Kv, Vv, row_scale, col_scale, dS, bq, out_scale, N, d, causal, sm_scale,
-               p_mode, round32, r0, r1, tile=TILE):
+               p_mode, round32, r0, r1, tile=TILE, with_lse=False):
     out = np.empty((r1 - r0, d), np.float64)
+    lse = np.empty(r1 - r0, np.float64) if with_lse else None
     _ok(lib().or_attn_core(_p(Qv), _p(Kv), _p(Vv), _p(row_scale), _p(col_scale), _p(dS), int(bq),
                            _p(out_scale), N, d, tile, int(causal), float(sm_scale), int(p_mode),
-                           int(round32), int(r0), int(r1), _p(out)), "attn_core")
-    return out
+                           int(round32), int(r0), int(r1), _p(out), _p(lse)), "attn_core")
+    return (out, lse) if with_lse else out
 
 
 def attention_sage_head(quant: Dict[str, np.ndarray], b: int, h: int, r0: int, r1: int, *,
-                        bq: int, bk: int, causal: bool, sm_scale: float, tile: int = TILE) -> np.ndarray:
+                        bq: int, bk: int, causal: bool, sm_scale: float, tile: int = TILE,
+                        with_lse: bool = False):
     """SageAttention2 Algorithm 1 (INT8 QK^T, E4M3 P~*448, FP8 PV, two-level FP32
-    accumulation, final / 448 * delta_V) for rows [r0, r1) of head (b, h)."""
+    accumulation, final / 448 * delta_V) for rows [r0, r1) of head (b, h).
+    with_lse: also the rows' log-sum-exp of the scores the algorithm uses (those
+    of the smoothed K; add lse_smooth_k_correction for the unsmoothed keys)."""
     Hq, Hkv = quant["q8"].shape[1], quant["k8"].shape[1]
     g = h // (Hq // Hkv)
     N, d = quant["q8"].shape[2], quant["q8"].shape[3]
@@ -266,7 +270,20 @@ def attention_sage_head(quant: Dict[str, np.ndarray], b: int, h: int, r0: int, r
     dS = np.ascontiguousarray(quant["dS"][b, h]) if "dS" in quant else None
     out_scale = np.ascontiguousarray(quant["s_v"][b, g], np.float64)
     return _attn_core(Qv, Kv, Vv, row_scale, col_scale, dS, bq, out_scale, N, d, causal, sm_scale,
-                      1, 1, r0, r1, tile)
+                      1, 1, r0, r1, tile, with_lse)
+
+
+def lse_smooth_k_correction(q, quant: Dict[str, np.ndarray], b: int, h: int, r0: int, r1: int, *,
+                            sm_scale: float) -> np.ndarray:
+    """Smooth K subtracts km from every key, which shifts row i's scores by the
+    constant sm_scale (Q_i . km): softmax is unchanged, the log-sum-exp is not.
+    Adding this (fp64) to the log-sum-exp of the smoothed scores gives the one
+    over the original keys (SageAttention2 note, "Smooth K" and its
+    "softmax invariance" remark).  km is zero without smooth K."""
+    Hq, Hkv = quant["q8"].shape[1], quant["k8"].shape[1]
+    g = h // (Hq // Hkv)
+    Q = np.asarray(_f32(q[b, h]), np.float64)[r0:r1]
+    return sm_scale * (Q @ quant["km"][b, g].astype(np.float64))
 
 
 def attention_exact_head(q, k, v, b: int, h: int, r0: int, r1: int, *, causal: bool, sm_scale: float):
@@ -284,7 +301,7 @@ def attention_exact_head(q, k, v, b: int, h: int, r0: int, r1: int, *, causal: b
 
 
 def attention_blocked_f64_head(q, k, v, b: int, h: int, r0: int, r1: int, *, causal: bool,
-                               sm_scale: float, tile: int = TILE):
+                               sm_scale: float, tile: int = TILE, with_lse: bool = False):
     """The oracle's blocked online softmax with identity codecs, all in fp64."""
     Hq, Hkv = q.shape[1], k.shape[1]
     g = h // (Hq // Hkv)
@@ -292,7 +309,7 @@ def attention_blocked_f64_head(q, k, v, b: int, h: int, r0: int, r1: int, *, cau
     K = np.ascontiguousarray(_f32(k[b, g]), np.float64)
     V = np.ascontiguousarray(_f32(v[b, g]), np.float64)
     N, d = Q.shape
-    return _attn_core(Q, K, V, None, None, None, 1, None, N, d, causal, sm_scale, 0, 0, r0, r1, tile)
+    return _attn_core(Q, K, V, None, None, None, 1, None, N, d, causal, sm_scale, 0, 0, r0, r1, tile, with_lse)
 
 
 # ---------------------------------------------------------------- NVFP4 (SageAttention3)

@@ -315,7 +315,7 @@ int or_attn_core(const double *Qv, const double *Kv, const double *Vv,
                  const float *dS, int bq, const double *out_scale,
                  int64_t N, int d, int tile, int causal, double sm_scale,
                  int p_mode, int round32,
-                 int64_t r0, int64_t r1, double *out)
+                 int64_t r0, int64_t r1, double *out, double *lse)
 {
     int64_t r, j0, c;
     int k;
@@ -399,6 +399,9 @@ int or_attn_core(const double *Qv, const double *Kv, const double *Vv,
             if (out_scale) o = RND(o * out_scale[k]);
             out[(r - r0) * d + k] = o;
         }
+        /* log-sum-exp of the row's scores S (natural log): m + ln l, where l
+           is the running sum of exp(S - m) over the visible keys */
+        if (lse) lse[r - r0] = (l > 0.0) ? m + log(l) : -INFINITY;
     }
     free(S); free(P); free(O); free(Ot);
     return 0;

@@ -26,7 +26,8 @@ int or_attn_core(const double *Qv, const double *Kv, const double *Vv,
                  const double *row_scale, const double *col_scale,
                  const float *dS, int bq, const double *out_scale,
                  int64_t N, int d, int tile, int causal, double sm_scale,
-                 int p_mode, int round32, int64_t r0, int64_t r1, double *out);
+                 int p_mode, int round32, int64_t r0, int64_t r1, double *out,
+                 double *lse /* NULL, or r1 - r0 log-sum-exps of the rows' scores */);
 int or_attn_naive_f64(const double *Q, const double *K, const double *V,
                       int64_t N, int d, int causal, double sm_scale,
                       int64_t r0, int64_t r1, double *out);

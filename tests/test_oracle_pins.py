@@ -379,3 +379,80 @@ def test_nvfp4_quant_properties():
     assert sf.shape == (3, 16)
     # groups run along tokens: group 2 covers rows 32..36 only
     assert t8[sf[2, 0]] == t8[oracle.e4m3_encode(np.array([np.abs(V[32:, 0]).max() / 6], np.float32))[0]]
+
+
+# ---------------------------------------------------------------- log-sum-exp
+def _lse_textbook(Q, K, sm_scale, causal):
+    """fp64 log-sum-exp of each row of sm_scale Q K^T (causal: keys <= row), via
+    scipy's logsumexp -- an independent routine."""
+    from scipy.special import logsumexp
+    S = (Q.astype(np.float64) @ K.astype(np.float64).T) * sm_scale
+    if causal:
+        S = np.where(np.tril(np.ones_like(S, dtype=bool)), S, -np.inf)
+    return logsumexp(S, axis=1)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("tile", [16, 32, 128])
+def test_oracle_lse_identity_codecs_equals_logsumexp(causal, tile):
+    """The blocked online softmax's m + ln l (identity codecs, fp64) is the
+    row log-sum-exp: pins the running-max / running-sum bookkeeping."""
+    g = torch.Generator().manual_seed(11)
+    N, d = 77, 64
+    q = torch.randn(1, 1, N, d, generator=g) * 2
+    k = torch.randn(1, 1, N, d, generator=g) * 2
+    v = torch.randn(1, 1, N, d, generator=g)
+    _, lse = oracle.attention_blocked_f64_head(q, k, v, 0, 0, 0, N, causal=causal, sm_scale=0.125,
+                                               tile=tile, with_lse=True)
+    ref = _lse_textbook(q[0, 0].numpy(), k[0, 0].numpy(), 0.125, causal)
+    np.testing.assert_allclose(lse, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_oracle_lse_zero_keys_is_log_of_visible_keys():
+    N, d = 40, 64
+    q = torch.randn(1, 1, N, d, generator=torch.Generator().manual_seed(3))
+    k = torch.zeros(1, 1, N, d)
+    v = torch.ones(1, 1, N, d)
+    for causal in (False, True):
+        _, lse = oracle.attention_blocked_f64_head(q, k, v, 0, 0, 0, N, causal=causal, sm_scale=0.3,
+                                                   tile=16, with_lse=True)
+        visible = np.arange(1, N + 1) if causal else np.full(N, N)
+        np.testing.assert_allclose(lse, np.log(visible), rtol=0, atol=1e-13)
+
+
+def test_oracle_lse_smooth_k_shift_identity():
+    """Shifting every key by a constant vector km shifts row i's scores by
+    sm_scale (Q_i . km): lse(K + km) = lse(K) + sm_scale Q km.  Inputs are small
+    dyadic values so that K + km is exact in fp32."""
+    g = torch.Generator().manual_seed(5)
+    N, d = 50, 64
+    q = torch.randint(-16, 17, (1, 1, N, d), generator=g).float() / 8
+    k = torch.randint(-16, 17, (1, 1, N, d), generator=g).float() / 8
+    km = torch.randint(-8, 9, (d,), generator=g).float() / 4
+    v = torch.randn(1, 1, N, d, generator=g)
+    sm = 0.125
+    _, lse_k = oracle.attention_blocked_f64_head(q, k, v, 0, 0, 0, N, causal=True, sm_scale=sm, with_lse=True)
+    _, lse_shift = oracle.attention_blocked_f64_head(q, k + km, v, 0, 0, 0, N, causal=True, sm_scale=sm,
+                                                     with_lse=True)
+    corr = sm * (q[0, 0].double().numpy() @ km.double().numpy())
+    np.testing.assert_allclose(lse_shift, lse_k + corr, rtol=1e-12, atol=1e-10)
+
+
+def test_oracle_sage_lse_with_correction_tracks_exact():
+    """The quantised pipeline's log-sum-exp (smoothed K) plus the smooth-K
+    correction lands on the exact fp64 log-sum-exp of the original scores; a
+    dropped or sign-flipped correction would be off by |sm_scale Q km|, which
+    the K bias of the prefill recipe makes several units large."""
+    from quantized_attention_block_b200 import workloads as W
+    ws = W.small_variant(W.get("prefill"), N=200, B=1, Hq=1, Hkv=1)
+    q, k, v = W.make_qkv(ws)
+    quant = oracle.quantize_sage(q, k, v, bq=ws.bq, bk=ws.bk, smooth_k=True, smooth_q=False)
+    _, lse = oracle.attention_sage_head(quant, 0, 0, 0, ws.N, bq=ws.bq, bk=ws.bk, causal=ws.causal,
+                                        sm_scale=ws.sm_scale, with_lse=True)
+    corr = oracle.lse_smooth_k_correction(q, quant, 0, 0, 0, ws.N, sm_scale=ws.sm_scale)
+    ref = _lse_textbook(q[0, 0].float().numpy(), k[0, 0].float().numpy(), ws.sm_scale, ws.causal)
+    err_with = np.abs(lse + corr - ref).max()      # the INT8 score quantisation error (K outliers)
+    err_without = np.abs(lse - ref).max()
+    err_flipped = np.abs(lse - corr - ref).max()
+    assert np.abs(corr).max() > 1.0  # the correction matters on this recipe
+    assert err_with < 0.5 and err_with < 0.05 * err_without and err_with < 0.05 * err_flipped
