@@ -97,6 +97,9 @@ typedef struct {
     float   *qbar;  /* [B, Hq,  Tm, d]  Q block means (NULL unless smooth_q)     */
     float   *dS;    /* [B, Hq,  Tm, Np] delta_S = qbar . gamma(K)^T (or NULL)     */
     int64_t  Np;
+    float   *qkm;   /* [B, Hq,  Np]     Q_i . km (fp32; zeros without smooth_k): the
+                                        constant by which smooth K shifts row i's
+                                        scores, sm_scale-free (log-sum-exp correction) */
 } sage_quant_view;
 
 /* Bytes of workspace the entry points below need for `p` (0 if p is invalid). */
@@ -141,6 +144,24 @@ SAGE_API sage_status sage_attn_fwd_quantized(const sage_quant_view *view, void *
 /* sage_quant_qkv followed by sage_attn_fwd_quantized (the whole forward). */
 SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, void *o, const sage_params *p,
                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sage_attn_fwd_quantized that also writes each row's log-sum-exp of the
+ * attention scores (the return_lse of the SageAttention API):
+ *   lse[b, h, i] = ln sum_j exp(S_ij) + sm_scale (Q_i . km)
+ * S are the scores the kernel uses (dequantised INT8 Q^K^T on the smoothed K,
+ * + delta_S, times sm_scale; causal: keys j <= i); the second term undoes the
+ * row-constant shift of smooth K (zero without it), so lse refers to the
+ * original keys.  lse: device fp32 [B, Hq, N], 4-byte aligned, caller-owned.
+ * SAGE_ERR_INVALID_ARG if lse is misaligned or the view lacks qkm.
+ */
+SAGE_API sage_status sage_attn_fwd_quantized_lse(const sage_quant_view *view, void *o, float *lse,
+                                                 const sage_params *p, void *stream);
+
+/* sage_quant_qkv followed by sage_attn_fwd_quantized_lse. */
+SAGE_API sage_status sage_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float *lse,
+                                       const sage_params *p, void *workspace, size_t workspace_bytes,
+                                       void *stream);
 
 /*
  * Bit-exactness probe of the INT8 tensor-core path: the raw INT32 tile

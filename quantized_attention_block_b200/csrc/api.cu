@@ -27,7 +27,7 @@ struct Dims {
 };
 
 struct Layout {
-  size_t q8, k8, v8t, s_q, s_k, s_v, km, ksum, vamax, kv_sync, kv_sync_end, qbar, dS, total;
+  size_t q8, k8, v8t, s_q, s_k, s_v, km, qkm, ksum, vamax, kv_sync, kv_sync_end, qbar, dS, total;
 };
 
 // 1: sage_quant_qkv always takes the two-pass K/V path (sage_debug_kv_quant_two_pass)
@@ -74,6 +74,7 @@ Layout make_layout(const sage_params* p, const Dims& d) {
   L.s_k = take(4 * (size_t)(d.B * d.Hkv * d.Tn));
   L.s_v = take(4 * (size_t)(d.B * d.Hkv * d.D));
   L.km = take(4 * (size_t)(d.B * d.Hkv * d.D));
+  L.qkm = take(4 * (size_t)(d.B * d.Hq * d.Np));
   // ksum, vamax, kv_sync consecutive: the one-read K/V kernel zeroes them with one memset
   L.ksum = take(8 * (size_t)(d.B * d.Hkv * d.D));
   L.vamax = take(4 * (size_t)(d.B * d.Hkv * d.D));
@@ -155,6 +156,7 @@ sage_status fill_view(const sage_params* p, const Dims& d, void* ws, sage_quant_
   v->qbar = p->smooth_q ? reinterpret_cast<float*>(base + L.qbar) : nullptr;
   v->dS = p->smooth_q ? reinterpret_cast<float*>(base + L.dS) : nullptr;
   v->Np = d.Np;
+  v->qkm = reinterpret_cast<float*>(base + L.qkm);
   return SAGE_OK;
 }
 
@@ -187,6 +189,8 @@ AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d
   a.n_qtiles = (int)(d.Np / kTile);
   const float sm = p->sm_scale > 0.0f ? p->sm_scale : 1.0f / std::sqrt((float)d.D);
   a.scale_log2 = (float)((double)sm * 1.4426950408889634);
+  a.sm_scale = sm;
+  a.qkm = v->qkm;
   a.s_q = v->s_q;
   a.s_k = v->s_k;
   a.s_v = v->s_v;
@@ -339,6 +343,7 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
   a.km = view->km;
   a.qbar = view->qbar;
   a.dS = view->dS;
+  a.qkm = view->qkm;
   a.ksum = reinterpret_cast<double*>(base + L.ksum);
   a.vamax = reinterpret_cast<unsigned*>(base + L.vamax);
   a.kv_sync = g_kv_two_pass ? nullptr : reinterpret_cast<int*>(base + L.kv_sync);
@@ -354,6 +359,11 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
 }
 
 sage_status sage_attn_fwd_quantized(const sage_quant_view* view, void* o, const sage_params* p, void* stream) {
+  return sage_attn_fwd_quantized_lse(view, o, nullptr, p, stream);
+}
+
+sage_status sage_attn_fwd_quantized_lse(const sage_quant_view* view, void* o, float* lse, const sage_params* p,
+                                        void* stream) {
   Dims d;
   sage_status s = check_params(p, &d);
   if (s != SAGE_OK) return s;
@@ -366,17 +376,24 @@ sage_status sage_attn_fwd_quantized(const sage_quant_view* view, void* o, const 
   if ((s = check_arch()) != SAGE_OK) return s;
   CUtensorMap mQ, mK, mV;
   if ((s = make_maps(view, d, &mQ, &mK, &mV)) != SAGE_OK) return s;
+  if (lse && (!view->qkm || (reinterpret_cast<uintptr_t>(lse) & 3u))) return SAGE_ERR_INVALID_ARG;
   AttnArgs a = attn_args(view, p, d);
   a.o = o;
+  a.lse = lse;
   return from_cuda(launch_attn_i8f8(a, mQ, mK, mV, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* o, const sage_params* p,
                           void* workspace, size_t workspace_bytes, void* stream) {
+  return sage_attn_fwd_lse(q, k, v, o, nullptr, p, workspace, workspace_bytes, stream);
+}
+
+sage_status sage_attn_fwd_lse(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const sage_params* p, void* workspace, size_t workspace_bytes, void* stream) {
   sage_quant_view view;
   sage_status s = sage_quant_qkv(q, k, v, p, workspace, workspace_bytes, &view, stream);
   if (s != SAGE_OK) return s;
-  return sage_attn_fwd_quantized(&view, o, p, stream);
+  return sage_attn_fwd_quantized_lse(&view, o, lse, p, stream);
 }
 
 sage_status sage_debug_qk_int32(const sage_quant_view* view, const sage_params* p, int32_t b, int32_t h,

@@ -83,8 +83,8 @@ struct Smem {
   static constexpr uint32_t kDS = 2 * 4 * 128 * 4;      // delta_S rows of one key tile: [tile][Q block (<= 4)][128]
   static constexpr uint32_t oDS = oP + 4 * kP;           // kStages
   static constexpr uint32_t oAlpha = oDS + kStages * kDS;  // float[tile][buffer][128]
-  static constexpr uint32_t oL = oAlpha + 4 * 128 * 4;   // float[2][128]
-  static constexpr uint32_t oBar = oL + 2 * 128 * 4;
+  static constexpr uint32_t oL = oAlpha + 4 * 128 * 4;   // float[2][128] l, then float[2][128] m
+  static constexpr uint32_t oBar = oL + 2 * 2 * 128 * 4;
   static constexpr uint32_t kNumBars = 1 + 3 * kStages + 2 + 4 + 4 + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = oTmem + 16 + 1024;  // + alignment slack
@@ -502,6 +502,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       m = m_new;
     }
     s_l[ti * 128 + row] = l;
+    s_l[256 + ti * 128 + row] = m;
     mbar_arrive(&bar.l_ready[ti]);
   } else {
     // ------------------------------------------------------------ correction + epilogue
@@ -614,6 +615,15 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       tc_fence_after();
       const float inv_l = 1.0f / s_l[i * 128 + row];
       const int64_t qrow = (int64_t)(2 * pr + i) * kTile + row;
+      if (a.lse != nullptr && qrow < a.N) {
+        // ln sum_j e^(S_ij) = (m + log2(l / 448)) ln 2 (m: running max of the
+        // log2-domain scores, l: sum of 448 2^(t - m)), plus the smooth-K shift
+        const float l = s_l[i * 128 + row], m = s_l[256 + i * 128 + row];
+        const int64_t bhq = (int64_t)(b * a.Hq + h);
+        a.lse[bhq * a.N + qrow] =
+            l > 0.0f ? (m + log2f(l) - kLog2_448) * 0.69314718055994531f + a.sm_scale * a.qkm[bhq * a.Np + qrow]
+                     : -INFINITY;
+      }
       const float* sv = a.s_v + (int64_t)(b * a.Hkv + g) * D;
       TO* out = reinterpret_cast<TO*>(a.o) + ((int64_t)(b * a.Hq + h) * a.N + qrow) * D;
       const uint32_t tO = tmem + 256 + D * i + lane_off;

@@ -27,6 +27,7 @@ struct QuantArgs {
   float* km;
   float* qbar;
   float* dS;
+  float* qkm;  // [B,Hq,Np] Q_i . km in fp32 (written by the Q kernel; zeros without smooth K)
   double* ksum;     // [B,Hkv,D] fp64 column sums of K
   unsigned* vamax;  // [B,Hkv,D] bit pattern of max |V| (non-negative floats order as uints);
                     // nullptr: the statistics pass skips V (NVFP4 path)
@@ -54,11 +55,14 @@ struct AttnArgs {
   int causal;
   int n_qtiles;
   float scale_log2;  // sm_scale * log2(e)
+  float sm_scale;
   const float* s_q;
   const float* s_k;
   const float* s_v;
   const float* dS;  // nullptr when smooth_q is off
   void* o;          // [B,Hq,N,D] bf16/fp16
+  float* lse;        // [B,Hq,N] natural-log log-sum-exp of the rows' scores, or nullptr
+  const float* qkm;  // [B,Hq,Np] Q_i . km (the smooth-K correction of lse / sm_scale)
   int out_fp16;
   int two_level;  // 1: fresh O_t per key tile + FP32 add on CUDA cores; 0: TMEM FP32 accumulator
   // NVFP4 scale blocks (1 KB per 128-row tile)

@@ -386,6 +386,28 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
     }
   }
   if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh)) return;
+  if (!IS_K && a.qkm != nullptr) {
+    // Q_i . km of every row of the tile (fp32), from the unshifted rows: the
+    // constant by which smooth K shifts row i's scores (log-sum-exp correction)
+    constexpr int CH = D / 8, RG = kThreads / CH;
+    const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+    const float* km = a.km + (int64_t)((bh / a.Hq) * a.Hkv + (bh % a.Hq) / (a.Hq / a.Hkv)) * D + ch * 8;
+    float kmc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) kmc[e] = km[e];
+#pragma unroll 4
+    for (int p = 0; p < kTile / RG; ++p) {
+      const int r = rg + p * RG;
+      float x[8];
+      lds8(sX + r * D + ch * 8, x);  // rows past N are zero
+      float dot = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dot = fmaf(x[e], kmc[e], dot);
+#pragma unroll
+      for (int o = CH / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if (ch == 0) a.qkm[(int64_t)bh * a.Np + r0 + r] = dot;
+    }
+  }
   if (!IS_K && SHIFT) block_means<T, D, BQ>(sX, s_sum, s_shift, bh, tile, a);
   __syncthreads();
   qk_encode<T, D, BQ, IS_K, SHIFT>(sX, s_shift, s_red, s_bmax, bh, tile, a);

@@ -28,7 +28,8 @@ EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized",
             "sage_status_string", "sage_attn_fwd_noalloc", "sage_debug_f8_accum_probe",
             "sage_nvfp4_workspace_bytes", "sage_quant_nvfp4", "sage_attn_fwd_nvfp4_quantized",
             "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4", "sage_debug_exp2_poly",
-            "sage_debug_kv_quant_two_pass", "sage_quant_kernel_count", "sage_quant_nvfp4_kernel_count")
+            "sage_debug_kv_quant_two_pass", "sage_quant_kernel_count", "sage_quant_nvfp4_kernel_count",
+            "sage_attn_fwd_quantized_lse", "sage_attn_fwd_lse")
 
 
 class SageError(RuntimeError):
@@ -52,7 +53,7 @@ class SageQuantView(ctypes.Structure):
     _fields_ = [("q8", ctypes.c_void_p), ("k8", ctypes.c_void_p), ("v8t", ctypes.c_void_p),
                 ("s_q", ctypes.c_void_p), ("s_k", ctypes.c_void_p), ("s_v", ctypes.c_void_p),
                 ("km", ctypes.c_void_p), ("qbar", ctypes.c_void_p), ("dS", ctypes.c_void_p),
-                ("Np", ctypes.c_int64)]
+                ("Np", ctypes.c_int64), ("qkm", ctypes.c_void_p)]
 
 
 class SageNvfp4View(ctypes.Structure):
@@ -78,6 +79,10 @@ def lib() -> ctypes.CDLL:
         L.sage_quant_qkv.argtypes = [vp, vp, vp, P, vp, ctypes.c_size_t, V, vp]
         L.sage_attn_fwd_quantized.argtypes = [V, vp, P, vp]
         L.sage_attn_fwd.argtypes = [vp, vp, vp, vp, P, vp, ctypes.c_size_t, vp]
+        L.sage_attn_fwd_quantized_lse.argtypes = [V, vp, vp, P, vp]
+        L.sage_attn_fwd_quantized_lse.restype = ctypes.c_int
+        L.sage_attn_fwd_lse.argtypes = [vp, vp, vp, vp, vp, P, vp, ctypes.c_size_t, vp]
+        L.sage_attn_fwd_lse.restype = ctypes.c_int
         L.sage_debug_qk_int32.argtypes = [V, P, i32, i32, i32, i32, vp, vp]
         L.sage_last_device_error.argtypes = [vp]
         L.sage_debug_bounded_wait.argtypes = [ctypes.c_uint32, vp]
@@ -168,6 +173,31 @@ def sage_attn_fwd(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = 
     return out
 
 
+def sage_attn_fwd_lse(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = None, smooth_k: bool = True,
+                      smooth_q: bool = False, bq: int = 128, bk: int = 64, pv_accum: int = PV_TWO_LEVEL,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None):
+    """sage_attn_fwd that also returns each row's log-sum-exp of the scores
+    (fp32 [B,Hq,N], natural log, for the original keys): (out, lse)."""
+    p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq, bk=bk,
+                    pv_accum=pv_accum)
+    if workspace is None:
+        workspace = alloc_workspace(p, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((p.B, p.Hq, p.N), dtype=torch.float32, device=q.device)
+    _check(lib().sage_attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), ctypes.byref(p),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)), "sage_attn_fwd_lse")
+    return out, lse
+
+
+def sage_attn_fwd_quantized_lse(view: SageQuantView, o: torch.Tensor, lse: torch.Tensor, p: SageParams,
+                                stream=None) -> None:
+    _check(lib().sage_attn_fwd_quantized_lse(ctypes.byref(view), _ptr(o), _ptr(lse), ctypes.byref(p),
+                                             _stream(stream)), "sage_attn_fwd_quantized_lse")
+
+
 def sage_debug_qk_int32(view: SageQuantView, p: SageParams, b: int, h: int, qtile: int, ktile: int,
                         stream=None) -> torch.Tensor:
     out = torch.empty((128, 128), dtype=torch.int32, device="cuda")
@@ -214,6 +244,7 @@ def view_tensors(view: SageQuantView, p: SageParams, workspace: torch.Tensor) ->
         "s_k": sl(view.s_k, 4 * B * Hkv * Tn, torch.float32, (B, Hkv, Tn)),
         "s_v": sl(view.s_v, 4 * B * Hkv * d, torch.float32, (B, Hkv, d)),
         "km": sl(view.km, 4 * B * Hkv * d, torch.float32, (B, Hkv, d)),
+        "qkm": sl(view.qkm, 4 * B * Hq * Np, torch.float32, (B, Hq, Np)),
     }
     if view.qbar:
         out["qbar"] = sl(view.qbar, 4 * B * Hq * Tm * d, torch.float32, (B, Hq, Tm, d))

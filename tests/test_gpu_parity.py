@@ -121,6 +121,39 @@ def test_attention_matches_oracle_elementwise(name, mode):
     assert ok, m
 
 
+LSE_CASES = ["prefill", "video", "gqa", "N127_causal", "N300_no_smooth_k", "N257_smoothq_causal_d128",
+             "N260_bq32_smoothq_gqa_causal", "N200_fp16_bq64_bk128"]
+
+
+@pytest.mark.parametrize("mode", list(PV_MODES))
+@pytest.mark.parametrize("name", LSE_CASES)
+def test_lse_matches_oracle(name, mode):
+    """Each row's log-sum-exp (return_lse) against the oracle's m + ln l of the
+    same quantised scores plus the smooth-K correction sm_scale Q.km (fp64):
+    within 1e-4 + 1e-5 |lse| (fp32 sums and the approximate exp2 / log2).
+    Asking for it leaves the output bit-identical."""
+    w = {**SMALL, **EDGE}[name]
+    q, k, v = W.make_qkv(w)
+    p, ws, view, (qd, kd, vd) = gpu_quant(w, q, k, v, PV_MODES[mode])
+    o1, o2 = torch.empty_like(qd), torch.empty_like(qd)
+    lse = torch.full((w.B, w.Hq, w.N), float("nan"), dtype=torch.float32, device="cuda")
+    sage.sage_attn_fwd_quantized(view, o1, p)
+    sage.sage_attn_fwd_quantized_lse(view, o2, lse, p)
+    torch.cuda.synchronize()
+    assert sage.sage_last_device_error() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    quant = oracle_quant(w, q, k, v)
+    got = lse.cpu().numpy().astype(np.float64)
+    sm = w.sm_scale if w.sm_scale else 1.0 / np.sqrt(w.d)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            _, l = oracle.attention_sage_head(quant, b, h, 0, w.N, bq=w.bq, bk=w.bk, causal=w.causal,
+                                              sm_scale=w.sm_scale, with_lse=True)
+            ref = l + oracle.lse_smooth_k_correction(q, quant, b, h, 0, w.N, sm_scale=sm)
+            err = np.abs(got[b, h] - ref)
+            assert np.all(err <= 1e-4 + 1e-5 * np.abs(ref)), (b, h, float(err.max()), int(np.argmax(err)))
+
+
 def test_pv_accumulation_modes_agree_closely():
     """The TMEM FP32 accumulator and the two-level scheme differ only in FP32
     rounding order (the accumulator keeps full FP32: see the probe test)."""
