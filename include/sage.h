@@ -76,6 +76,9 @@ typedef struct {
                                     TMEM accumulator, rescaled on CUDA cores only for
                                     rows whose max grew (tcgen05 keeps full FP32 in
                                     the accumulator: see sage_debug_f8_accum_probe) */
+    int32_t return_lse;        /* 1: sage_quant_qkv also computes Q_i . km (view->qkm) so
+                                  that sage_attn_fwd_quantized_lse can write the
+                                  log-sum-exp; 0: view->qkm is NULL (INT8/FP8 path) */
 } sage_params;
 
 enum { SAGE_PV_TWO_LEVEL = 0, SAGE_PV_TMEM_FP32 = 1 };
@@ -99,7 +102,8 @@ typedef struct {
     int64_t  Np;
     float   *qkm;   /* [B, Hq,  Np]     Q_i . km (fp32; zeros without smooth_k): the
                                         constant by which smooth K shifts row i's
-                                        scores, sm_scale-free (log-sum-exp correction) */
+                                        scores, sm_scale-free (log-sum-exp correction);
+                                        NULL unless p->return_lse */
 } sage_quant_view;
 
 /* Bytes of workspace the entry points below need for `p` (0 if p is invalid). */
@@ -153,12 +157,14 @@ SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, 
  * + delta_S, times sm_scale; causal: keys j <= i); the second term undoes the
  * row-constant shift of smooth K (zero without it), so lse refers to the
  * original keys.  lse: device fp32 [B, Hq, N], 4-byte aligned, caller-owned.
- * SAGE_ERR_INVALID_ARG if lse is misaligned or the view lacks qkm.
+ * SAGE_ERR_INVALID_ARG if lse is misaligned or the view lacks qkm (the view
+ * must come from sage_quant_qkv with p->return_lse = 1).
  */
 SAGE_API sage_status sage_attn_fwd_quantized_lse(const sage_quant_view *view, void *o, float *lse,
                                                  const sage_params *p, void *stream);
 
-/* sage_quant_qkv followed by sage_attn_fwd_quantized_lse. */
+/* sage_quant_qkv followed by sage_attn_fwd_quantized_lse (return_lse is
+ * taken as 1 whatever p says). */
 SAGE_API sage_status sage_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float *lse,
                                        const sage_params *p, void *workspace, size_t workspace_bytes,
                                        void *stream);

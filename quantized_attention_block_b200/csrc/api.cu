@@ -45,6 +45,7 @@ sage_status check_params(const sage_params* p, Dims* d) {
     return SAGE_ERR_INVALID_ARG;
   if (std::isnan(p->sm_scale) || std::isinf(p->sm_scale)) return SAGE_ERR_INVALID_ARG;
   if (p->pv_accum != SAGE_PV_TWO_LEVEL && p->pv_accum != SAGE_PV_TMEM_FP32) return SAGE_ERR_INVALID_ARG;
+  if (p->return_lse != 0 && p->return_lse != 1) return SAGE_ERR_INVALID_ARG;
   d->B = p->B;
   d->Hq = p->Hq;
   d->Hkv = p->Hkv;
@@ -156,7 +157,7 @@ sage_status fill_view(const sage_params* p, const Dims& d, void* ws, sage_quant_
   v->qbar = p->smooth_q ? reinterpret_cast<float*>(base + L.qbar) : nullptr;
   v->dS = p->smooth_q ? reinterpret_cast<float*>(base + L.dS) : nullptr;
   v->Np = d.Np;
-  v->qkm = reinterpret_cast<float*>(base + L.qkm);
+  v->qkm = p->return_lse ? reinterpret_cast<float*>(base + L.qkm) : nullptr;
   return SAGE_OK;
 }
 
@@ -390,10 +391,13 @@ sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* o, 
 
 sage_status sage_attn_fwd_lse(const void* q, const void* k, const void* v, void* o, float* lse,
                               const sage_params* p, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!p) return SAGE_ERR_INVALID_ARG;
+  sage_params pl = *p;
+  pl.return_lse = lse ? 1 : 0;
   sage_quant_view view;
-  sage_status s = sage_quant_qkv(q, k, v, p, workspace, workspace_bytes, &view, stream);
+  sage_status s = sage_quant_qkv(q, k, v, &pl, workspace, workspace_bytes, &view, stream);
   if (s != SAGE_OK) return s;
-  return sage_attn_fwd_quantized_lse(&view, o, lse, p, stream);
+  return sage_attn_fwd_quantized_lse(&view, o, lse, &pl, stream);
 }
 
 sage_status sage_debug_qk_int32(const sage_quant_view* view, const sage_params* p, int32_t b, int32_t h,

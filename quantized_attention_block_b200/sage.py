@@ -43,7 +43,7 @@ class SageParams(ctypes.Structure):
                 ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("sm_scale", ctypes.c_float), ("smooth_k", ctypes.c_int32),
                 ("smooth_q", ctypes.c_int32), ("bq", ctypes.c_int32), ("bk", ctypes.c_int32),
-                ("pv_accum", ctypes.c_int32)]
+                ("pv_accum", ctypes.c_int32), ("return_lse", ctypes.c_int32)]
 
 
 PV_TWO_LEVEL, PV_TMEM_FP32 = 0, 1
@@ -121,12 +121,12 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> int:
 
 def make_params(q: torch.Tensor, k: torch.Tensor, *, causal: bool = False, sm_scale: Optional[float] = None,
                 smooth_k: bool = True, smooth_q: bool = False, bq: int = 128, bk: int = 64,
-                pv_accum: int = PV_TWO_LEVEL) -> SageParams:
+                pv_accum: int = PV_TWO_LEVEL, return_lse: bool = False) -> SageParams:
     """Parameters for HND tensors q [B, Hq, N, d], k [B, Hkv, N, d]."""
     B, Hq, N, d = q.shape
     dt = {torch.bfloat16: 0, torch.float16: 1}.get(q.dtype, -1)
     return SageParams(B, Hq, k.shape[1], N, d, dt, int(causal), float(sm_scale if sm_scale else 0.0),
-                      int(smooth_k), int(smooth_q), bq, bk, int(pv_accum))
+                      int(smooth_k), int(smooth_q), bq, bk, int(pv_accum), int(return_lse))
 
 
 def workspace_bytes(p: SageParams) -> int:
@@ -244,8 +244,9 @@ def view_tensors(view: SageQuantView, p: SageParams, workspace: torch.Tensor) ->
         "s_k": sl(view.s_k, 4 * B * Hkv * Tn, torch.float32, (B, Hkv, Tn)),
         "s_v": sl(view.s_v, 4 * B * Hkv * d, torch.float32, (B, Hkv, d)),
         "km": sl(view.km, 4 * B * Hkv * d, torch.float32, (B, Hkv, d)),
-        "qkm": sl(view.qkm, 4 * B * Hq * Np, torch.float32, (B, Hq, Np)),
     }
+    if view.qkm:
+        out["qkm"] = sl(view.qkm, 4 * B * Hq * Np, torch.float32, (B, Hq, Np))
     if view.qbar:
         out["qbar"] = sl(view.qbar, 4 * B * Hq * Tm * d, torch.float32, (B, Hq, Tm, d))
         out["dS"] = sl(view.dS, 4 * B * Hq * Tm * Np, torch.float32, (B, Hq, Tm, Np))

@@ -134,7 +134,11 @@ def test_lse_matches_oracle(name, mode):
     Asking for it leaves the output bit-identical."""
     w = {**SMALL, **EDGE}[name]
     q, k, v = W.make_qkv(w)
-    p, ws, view, (qd, kd, vd) = gpu_quant(w, q, k, v, PV_MODES[mode])
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    p = sage.make_params(qd, kd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k, smooth_q=w.smooth_q,
+                         bq=w.bq, bk=w.bk, pv_accum=PV_MODES[mode], return_lse=True)
+    ws = sage.alloc_workspace(p)
+    view = sage.sage_quant_qkv(qd, kd, vd, p, ws)
     o1, o2 = torch.empty_like(qd), torch.empty_like(qd)
     lse = torch.full((w.B, w.Hq, w.N), float("nan"), dtype=torch.float32, device="cuda")
     sage.sage_attn_fwd_quantized(view, o1, p)
@@ -152,6 +156,21 @@ def test_lse_matches_oracle(name, mode):
             ref = l + oracle.lse_smooth_k_correction(q, quant, b, h, 0, w.N, sm_scale=sm)
             err = np.abs(got[b, h] - ref)
             assert np.all(err <= 1e-4 + 1e-5 * np.abs(ref)), (b, h, float(err.max()), int(np.argmax(err)))
+    # the one-call form gives the same bytes
+    o3, lse3 = sage.sage_attn_fwd_lse(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k,
+                                      smooth_q=w.smooth_q, bq=w.bq, bk=w.bk, pv_accum=PV_MODES[mode])
+    torch.cuda.synchronize()
+    assert torch.equal(o3.view(torch.int16), o2.view(torch.int16)) and torch.equal(lse3, lse)
+
+
+def test_lse_needs_return_lse_at_quantisation():
+    w = SMALL["prefill"]
+    q, k, v = W.make_qkv(w)
+    p, ws, view, (qd, kd, vd) = gpu_quant(w, q, k, v)
+    assert not view.qkm
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
+    with pytest.raises(sage.SageError):
+        sage.sage_attn_fwd_quantized_lse(view, torch.empty_like(qd), lse, p)
 
 
 def test_pv_accumulation_modes_agree_closely():
