@@ -79,7 +79,12 @@ typedef struct {
     int32_t return_lse;        /* 1: sage_quant_qkv also computes Q_i . km (view->qkm) so
                                   that sage_attn_fwd_quantized_lse can write the
                                   log-sum-exp; 0: view->qkm is NULL (INT8/FP8 path) */
+    int32_t layout;            /* sage_layout of q, k, v and o: SAGE_HND [B, H, N, d] or
+                                  SAGE_NHD [B, N, H, d] (the quantised tensors in the
+                                  workspace and lse are always head-major) */
 } sage_params;
+
+typedef enum { SAGE_HND = 0, SAGE_NHD = 1 } sage_layout;
 
 enum { SAGE_PV_TWO_LEVEL = 0, SAGE_PV_TMEM_FP32 = 1 };
 

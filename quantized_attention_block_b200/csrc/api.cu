@@ -46,6 +46,7 @@ sage_status check_params(const sage_params* p, Dims* d) {
   if (std::isnan(p->sm_scale) || std::isinf(p->sm_scale)) return SAGE_ERR_INVALID_ARG;
   if (p->pv_accum != SAGE_PV_TWO_LEVEL && p->pv_accum != SAGE_PV_TMEM_FP32) return SAGE_ERR_INVALID_ARG;
   if (p->return_lse != 0 && p->return_lse != 1) return SAGE_ERR_INVALID_ARG;
+  if (p->layout != SAGE_HND && p->layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
   d->B = p->B;
   d->Hq = p->Hq;
   d->Hkv = p->Hkv;
@@ -132,14 +133,16 @@ bool map_2d_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
 
 // [B*H][N][D] bf16/fp16 input as a 3D tensor (box 1 x 128 x D, no swizzle):
 // a tile that runs past N reads zeros.
-bool map_3d_input(CUtensorMap* m, const void* base, uint64_t D, uint64_t N, uint64_t BH) {
+// A caller's 16-bit input as a 4D (D, N, H, B) tensor whose strides encode its
+// layout (HND: [B, H, N, D]; NHD: [B, N, H, D]); box D x 128 x 1 x 1.
+bool map_input(CUtensorMap* m, const void* base, uint64_t D, uint64_t N, uint64_t H, uint64_t B, int nhd) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[3] = {D, N, BH};
-  const cuuint64_t strides[2] = {D * 2, N * D * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)D, kTile, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  const cuuint64_t dims[4] = {D, N, H, B};
+  const cuuint64_t strides[3] = {(nhd ? H * D : D) * 2, (nhd ? D : N * D) * 2, H * N * D * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)D, kTile, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -174,6 +177,14 @@ sage_status make_maps(const sage_quant_view* v, const Dims& d, CUtensorMap* mQ, 
   return SAGE_OK;
 }
 
+// element strides of the caller's o [B, Hq, N, d] (HND) or [B, N, Hq, d] (NHD)
+void set_out_strides(AttnArgs* a, const sage_params* p, const Dims& d) {
+  const int64_t D = d.D, N = d.N, Hq = d.Hq;
+  a->o_bs = Hq * N * D;
+  a->o_hs = p->layout == SAGE_NHD ? D : N * D;
+  a->o_rs = p->layout == SAGE_NHD ? Hq * D : D;
+}
+
 AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d) {
   AttnArgs a{};
   a.B = (int)d.B;
@@ -197,6 +208,7 @@ AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d
   a.s_v = v->s_v;
   a.dS = p->smooth_q ? v->dS : nullptr;
   a.out_fp16 = p->dtype == SAGE_FP16;
+  set_out_strides(&a, p, d);
   a.two_level = p->pv_accum == SAGE_PV_TWO_LEVEL;
   return a;
 }
@@ -288,6 +300,7 @@ AttnArgs attn_args_f4(const sage_nvfp4_view* v, const sage_params* p, const Dims
   a.scale_log2 = (float)((double)sm * 1.4426950408889634);
   a.dS = p->smooth_q ? v->dS : nullptr;
   a.out_fp16 = p->dtype == SAGE_FP16;
+  set_out_strides(&a, p, d);
   a.sfq = v->sfq;
   a.sfk = v->sfk;
   a.sfv = v->sfv;
@@ -335,6 +348,7 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
   a.bk = p->bk;
   a.smooth_k = p->smooth_k;
   a.smooth_q = p->smooth_q;
+  a.nhd = p->layout;
   a.q8 = view->q8;
   a.k8 = view->k8;
   a.v8t = view->v8t;
@@ -352,9 +366,9 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
   QuantMaps m;
   if (!map_2d_u8(&m.vt, view->v8t, (uint64_t)d.Np, (uint64_t)(d.B * d.Hkv * d.D), kTile, (uint32_t)d.D,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map_3d_input(&m.q, q, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hq)) ||
-      !map_3d_input(&m.k, k, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)) ||
-      !map_3d_input(&m.v, v, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)))
+      !map_input(&m.q, q, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)d.Hq, (uint64_t)d.B, p->layout) ||
+      !map_input(&m.k, k, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)d.Hkv, (uint64_t)d.B, p->layout) ||
+      !map_input(&m.v, v, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)d.Hkv, (uint64_t)d.B, p->layout))
     return SAGE_ERR_CUDA;
   return from_cuda(launch_quant(a, m, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));
 }
@@ -455,6 +469,7 @@ sage_status sage_quant_nvfp4(const void* q, const void* k, const void* v, const 
   a.bk = p->bk;
   a.smooth_k = p->smooth_k;
   a.smooth_q = p->smooth_q;
+  a.nhd = p->layout;
   a.km = view->km;
   a.qbar = view->qbar;
   a.dS = view->dS;
@@ -468,9 +483,9 @@ sage_status sage_quant_nvfp4(const void* q, const void* k, const void* v, const 
   a.kv_sync = g_kv_two_pass ? nullptr : reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + L.kv_sync);
   a.kv_zero_bytes = L.kv_sync_end - L.ksum;
   QuantMaps m;
-  if (!map_3d_input(&m.q, q, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hq)) ||
-      !map_3d_input(&m.k, k, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)) ||
-      !map_3d_input(&m.v, v, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)(d.B * d.Hkv)))
+  if (!map_input(&m.q, q, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)d.Hq, (uint64_t)d.B, p->layout) ||
+      !map_input(&m.k, k, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)d.Hkv, (uint64_t)d.B, p->layout) ||
+      !map_input(&m.v, v, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)d.Hkv, (uint64_t)d.B, p->layout))
     return SAGE_ERR_CUDA;
   m.vt = m.v;  // unused on this path
   return from_cuda(launch_quant_nvfp4(a, m, p->dtype == SAGE_FP16, static_cast<cudaStream_t>(stream)));

@@ -122,7 +122,9 @@ struct Bars {
   uint64_t* mma_done;  // all tensor-core work of the CTA retired (one commit at the end)
 };
 
-template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO>
+// LSE: also write each row's log-sum-exp (a separate instance, so that kernels
+// without it carry none of its code)
+template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO, bool LSE>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -502,7 +504,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       m = m_new;
     }
     s_l[ti * 128 + row] = l;
-    s_l[256 + ti * 128 + row] = m;
+    if (LSE) s_l[256 + ti * 128 + row] = m;
     mbar_arrive(&bar.l_ready[ti]);
   } else {
     // ------------------------------------------------------------ correction + epilogue
@@ -615,7 +617,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       tc_fence_after();
       const float inv_l = 1.0f / s_l[i * 128 + row];
       const int64_t qrow = (int64_t)(2 * pr + i) * kTile + row;
-      if (a.lse != nullptr && qrow < a.N) {
+      if (LSE && qrow < a.N) {
         // ln sum_j e^(S_ij) = (m + log2(l / 448)) ln 2 (m: running max of the
         // log2-domain scores, l: sum of 448 2^(t - m)), plus the smooth-K shift
         const float l = s_l[i * 128 + row], m = s_l[256 + i * 128 + row];
@@ -625,7 +627,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                      : -INFINITY;
       }
       const float* sv = a.s_v + (int64_t)(b * a.Hkv + g) * D;
-      TO* out = reinterpret_cast<TO*>(a.o) + ((int64_t)(b * a.Hq + h) * a.N + qrow) * D;
+      // row qrow of head (b, h): one formula for either layout (strides from the host)
+      TO* out = reinterpret_cast<TO*>(a.o) + b * a.o_bs + h * a.o_hs + qrow * a.o_rs;
       const uint32_t tO = tmem + 256 + D * i + lane_off;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
@@ -841,7 +844,8 @@ __global__ void bounded_wait_probe_kernel() {
 template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO>
 cudaError_t launch_attn_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                           cudaStream_t st) {
-  auto kern = attn_i8f8_kernel<D, CAUSAL, HAS_DS, TWO_LEVEL, TO>;
+  auto kern = a.lse ? attn_i8f8_kernel<D, CAUSAL, HAS_DS, TWO_LEVEL, TO, true>
+                    : attn_i8f8_kernel<D, CAUSAL, HAS_DS, TWO_LEVEL, TO, false>;
   const int smem = (int)Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

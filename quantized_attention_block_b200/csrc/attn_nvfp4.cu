@@ -524,7 +524,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
       tc_fence_after();
       const float f = s_l[i * 128 + row];
       const int64_t qrow = (int64_t)(2 * pr + i) * kTile + row;
-      TO* out = reinterpret_cast<TO*>(a.o) + ((int64_t)bh * a.N + qrow) * 128;
+      // row qrow of head (b, h): one formula for either layout (strides from the host)
+      TO* out = reinterpret_cast<TO*>(a.o) + b * a.o_bs + h * a.o_hs + qrow * a.o_rs;
       const uint32_t tA = tmem + kColA + 128 * i + lane_off;
 #pragma unroll
       for (int c = 0; c < 128; c += 32) {

@@ -9,6 +9,14 @@ namespace sage {
 
 constexpr int kTile = 128;  // attention tile: 128 Q rows x 128 keys
 
+// Element offset of row n of head bh (= b H + h) in a caller tensor of H heads,
+// N rows and D channels: [B, H, N, D] (HND) or [B, N, H, D] (NHD, nhd = 1).
+__host__ __device__ inline int64_t row_offset(int64_t bh, int64_t n, int H, int64_t N, int D, int nhd) {
+  return nhd ? (((bh / H) * N + n) * H + bh % H) * D : (bh * N + n) * D;
+}
+// elements between consecutive rows of one head
+__host__ __device__ inline int64_t row_stride(int H, int D, int nhd) { return nhd ? (int64_t)H * D : (int64_t)D; }
+
 struct QuantArgs {
   const void* q;  // [B,Hq,N,D] bf16/fp16
   const void* k;  // [B,Hkv,N,D]
@@ -17,6 +25,7 @@ struct QuantArgs {
   int64_t Np;
   int Tm, Tn, bq, bk;
   int smooth_k, smooth_q;
+  int nhd;  // q, k, v are [B, N, H, D] (else [B, H, N, D])
   // outputs / scratch (workspace)
   int8_t* q8;
   int8_t* k8;
@@ -60,7 +69,8 @@ struct AttnArgs {
   const float* s_k;
   const float* s_v;
   const float* dS;  // nullptr when smooth_q is off
-  void* o;          // [B,Hq,N,D] bf16/fp16
+  void* o;          // [B,Hq,N,D] bf16/fp16 ([B,N,Hq,D] when the caller's layout is NHD)
+  int64_t o_bs, o_hs, o_rs;  // element strides of o between batches, heads and rows
   float* lse;        // [B,Hq,N] natural-log log-sum-exp of the rows' scores, or nullptr
   const float* qkm;  // [B,Hq,Np] Q_i . km (the smooth-K correction of lse / sm_scale)
   int out_fp16;
@@ -74,8 +84,9 @@ struct AttnArgs {
   int32_t* probe_out;
 };
 
-// TMA maps of the preprocessing: the bf16/fp16 inputs as 3D [B*H][N][D] tensors
-// (box 1 x 128 x D) and the transposed E4M3 V output v8t (box D x 128 bytes).
+// TMA maps of the preprocessing: the bf16/fp16 inputs as 4D (D, N, H, B) tensors
+// with the caller's layout in the strides (box D x 128 x 1 x 1), and the
+// transposed E4M3 V output v8t (box D x 128 bytes).
 struct QuantMaps {
   CUtensorMap q, k, v, vt;
 };

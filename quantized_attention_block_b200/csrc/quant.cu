@@ -151,19 +151,20 @@ __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
   const int64_t r0 = (int64_t)blockIdx.x * kStatRows;
   const int64_t r1 = (r0 + kStatRows < (int64_t)a.N) ? r0 + kStatRows : (int64_t)a.N;
   const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
-  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
-  const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)bg * a.N * D;
+  const int64_t rs = row_stride(a.Hkv, D, a.nhd);
+  const T* K = reinterpret_cast<const T*>(a.k) + row_offset(bg, 0, a.Hkv, a.N, D, a.nhd);
+  const T* V = reinterpret_cast<const T*>(a.v) + row_offset(bg, 0, a.Hkv, a.N, D, a.nhd);
   double ks[8];
   float va[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) { ks[e] = 0.0; va[e] = 0.0f; }
   for (int64_t r = r0 + rg; r < r1; r += RG) {
     float x[8];
-    load8<T>(K + r * D + ch * 8, x);
+    load8<T>(K + r * rs + ch * 8, x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) ks[e] += (double)x[e];
     if (a.vamax) {
-      load8<T>(V + r * D + ch * 8, x);
+      load8<T>(V + r * rs + ch * 8, x);
 #pragma unroll
       for (int e = 0; e < 8; ++e) va[e] = fmaxf(va[e], fabsf(x[e]));
     }
@@ -186,11 +187,11 @@ __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
 
 // ---------------------------------------------------------------------------
 // Pass 2: one 128-row tile of Q, K or V per CTA.  The tile arrives in shared
-// memory by one TMA load (3D map [B*H][N][D]; rows past N read as zeros), so
+// memory by one TMA load (4D map (D, N, H, B); rows past N read as zeros), so
 // the registers hold no tile and several CTAs per SM keep HBM busy; the
 // threads then sweep the tile in shared memory (block sums, block max, codes).
 template <typename T, int D>
-__device__ __forceinline__ bool load_tile(T* dst, const CUtensorMap* map, uint64_t* bar, int row0, int bh) {
+__device__ __forceinline__ bool load_tile(T* dst, const CUtensorMap* map, uint64_t* bar, int row0, int bh, int H) {
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     mbar_fence_init();
@@ -198,7 +199,7 @@ __device__ __forceinline__ bool load_tile(T* dst, const CUtensorMap* map, uint64
   __syncthreads();
   if (threadIdx.x == 0) {
     mbar_expect_tx(bar, kTile * D * (uint32_t)sizeof(T));
-    tma_load_3d(dst, map, bar, 0, row0, bh);
+    tma_load_4d(dst, map, bar, 0, row0, bh % H, bh / H);
   }
   return mbar_wait(bar, 0);
 }
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
       for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = 0.0f;
     }
   }
-  if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh)) return;
+  if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh, IS_K ? a.Hkv : a.Hq)) return;
   if (!IS_K && a.qkm != nullptr) {
     // Q_i . km of every row of the tile (fp32), from the unshifted rows: the
     // constant by which smooth K shifts row i's scores (log-sum-exp correction)
@@ -475,7 +476,7 @@ __global__ void __launch_bounds__(kThreads)
     s_sv[c] = sv;
     if (tile == 0) a.s_v[(int64_t)bg * D + c] = sv;
   }
-  if (!load_tile<T, D>(sV, &tmX, &bar, (int)r0, bg)) return;
+  if (!load_tile<T, D>(sV, &tmX, &bar, (int)r0, bg, a.Hkv)) return;
   v_encode<T, D>(sV, sVt, s_sv, &tmVt, tile, bg);
 }
 
@@ -549,7 +550,7 @@ __global__ void __launch_bounds__(kThreads)
   const int grp = s_item / tiles, tile = s_item % tiles;
   const int bh = grp >> 1;
   const bool is_v = (grp & 1) != 0;
-  if (!load_tile<T, D>(sX, is_v ? &tmV : &tmK, &bar, tile * kTile, bh)) return;
+  if (!load_tile<T, D>(sX, is_v ? &tmV : &tmK, &bar, tile * kTile, bh, a.Hkv)) return;
   if (!is_v && !SMOOTH_K) {  // km = 0: nothing to wait for
     if (tile == 0 && threadIdx.x < D) a.km[(int64_t)bh * D + threadIdx.x] = 0.0f;
     qk_encode<T, D, BK, true, false>(sX, s_shift, s_red, s_bmax, bh, tile, a);
@@ -717,7 +718,8 @@ __global__ void __launch_bounds__(kThreads, 2) delta_s_tc_kernel(QuantArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  const T* K = reinterpret_cast<const T*>(a.k) + ((int64_t)bg * a.N + r0) * D;
+  const T* K = reinterpret_cast<const T*>(a.k) + row_offset(bg, r0, a.Hkv, a.N, D, a.nhd);
+  const int64_t krs = row_stride(a.Hkv, D, a.nhd);
   const float* km = a.km + (int64_t)bg * D;
   const float* qb = a.qbar + (int64_t)bh * a.Tm * D;
   float* out = a.dS + (int64_t)bh * a.Tm * a.Np + r0;
@@ -742,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 2) delta_s_tc_kernel(QuantArgs a) {
 #pragma unroll
     for (int it = 0; it < ITA; ++it) {
       const int r = (threadIdx.x + it * kThreads) / G8;
-      ka[it] = (load_a && r < valid) ? __ldg(reinterpret_cast<const uint4*>(K + (int64_t)r * D + pc0 + cl))
+      ka[it] = (load_a && r < valid) ? __ldg(reinterpret_cast<const uint4*>(K + (int64_t)r * krs + pc0 + cl))
                                      : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll

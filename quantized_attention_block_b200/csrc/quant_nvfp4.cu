@@ -66,14 +66,15 @@ __global__ void __launch_bounds__(kThreads) k_quant_nvfp4_kernel(QuantArgs a) {
     if (tile == 0) a.km[(int64_t)bg * D + c] = km;
   }
   __syncthreads();
-  const T* K = reinterpret_cast<const T*>(a.k) + (int64_t)bg * a.N * D;
+  const T* K = reinterpret_cast<const T*>(a.k) + row_offset(bg, 0, a.Hkv, a.N, D, a.nhd);
+  const int64_t rs = row_stride(a.Hkv, D, a.nhd);
   uint8_t* k4 = a.k4 + ((int64_t)bg * a.Np + r0) * (D / 2);
 #pragma unroll 2
   for (int p = 0; p < NP; ++p) {
     const int r = rg + p * RG;
     float x[8];
     if (r < valid) {
-      load8<T>(K + (r0 + r) * D + ch * 8, x);
+      load8<T>(K + (r0 + r) * rs + ch * 8, x);
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], s_km[ch * 8 + e]);
     } else {
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(kThreads) q_quant_nvfp4_kernel(const __grid_co
   __shared__ uint64_t bar;
   const int bh = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
-  if (!load_tile<T, D>(sX, &tmQ, &bar, (int)r0, bh)) return;
+  if (!load_tile<T, D>(sX, &tmQ, &bar, (int)r0, bh, a.Hq)) return;
   if (SHIFT) block_means<T, D, BQ>(sX, s_sum, s_mean, bh, tile, a);
   __syncthreads();
   nvfp4_encode_tile<T, BQ>(sX, SHIFT ? s_mean : nullptr, s_sf, rows_valid(a.N, r0, kTile),
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(kThreads) k_fused_nvfp4_kernel(const __grid_co
   if (threadIdx.x == 0) s_item = atomicAdd(a.kv_sync, 1);
   __syncthreads();
   const int bg = s_item / tiles, tile = s_item % tiles;
-  if (!load_tile<T, D>(sX, &tmK, &bar, tile * kTile, bg)) return;
+  if (!load_tile<T, D>(sX, &tmK, &bar, tile * kTile, bg, a.Hkv)) return;
   if constexpr (SMOOTH_K) {
     const int ch = threadIdx.x % CH, rg = threadIdx.x / CH, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     double cs[8];
@@ -227,12 +228,13 @@ __global__ void __launch_bounds__(kThreads) v_quant_nvfp4_kernel(QuantArgs a) {
   const int64_t r0 = (int64_t)tile * kTile;
   const int valid = rows_valid(a.N, r0, kTile);
   const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
-  const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)bg * a.N * D;
+  const T* V = reinterpret_cast<const T*>(a.v) + row_offset(bg, 0, a.Hkv, a.N, D, a.nhd);
+  const int64_t rs = row_stride(a.Hkv, D, a.nhd);
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int r = rg + p * RG;
     uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (r < valid) u = __ldg(reinterpret_cast<const uint4*>(V + (r0 + r) * D + ch * 8));
+    if (r < valid) u = __ldg(reinterpret_cast<const uint4*>(V + (r0 + r) * rs + ch * 8));
     *reinterpret_cast<uint4*>(sV + r * kPitch + ch * 8) = u;
   }
   __syncthreads();

@@ -43,10 +43,11 @@ class SageParams(ctypes.Structure):
                 ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("sm_scale", ctypes.c_float), ("smooth_k", ctypes.c_int32),
                 ("smooth_q", ctypes.c_int32), ("bq", ctypes.c_int32), ("bk", ctypes.c_int32),
-                ("pv_accum", ctypes.c_int32), ("return_lse", ctypes.c_int32)]
+                ("pv_accum", ctypes.c_int32), ("return_lse", ctypes.c_int32), ("layout", ctypes.c_int32)]
 
 
 PV_TWO_LEVEL, PV_TMEM_FP32 = 0, 1
+LAYOUTS = {"HND": 0, "NHD": 1}
 
 
 class SageQuantView(ctypes.Structure):
@@ -121,12 +122,20 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> int:
 
 def make_params(q: torch.Tensor, k: torch.Tensor, *, causal: bool = False, sm_scale: Optional[float] = None,
                 smooth_k: bool = True, smooth_q: bool = False, bq: int = 128, bk: int = 64,
-                pv_accum: int = PV_TWO_LEVEL, return_lse: bool = False) -> SageParams:
-    """Parameters for HND tensors q [B, Hq, N, d], k [B, Hkv, N, d]."""
-    B, Hq, N, d = q.shape
+                pv_accum: int = PV_TWO_LEVEL, return_lse: bool = False, tensor_layout: str = "HND") -> SageParams:
+    """Parameters for q [B, Hq, N, d], k [B, Hkv, N, d] (tensor_layout "HND") or
+    q [B, N, Hq, d], k [B, N, Hkv, d] ("NHD")."""
+    if tensor_layout not in LAYOUTS:
+        raise ValueError(f"tensor_layout must be one of {sorted(LAYOUTS)}")
+    if tensor_layout == "HND":
+        B, Hq, N, d = q.shape
+        Hkv = k.shape[1]
+    else:
+        B, N, Hq, d = q.shape
+        Hkv = k.shape[2]
     dt = {torch.bfloat16: 0, torch.float16: 1}.get(q.dtype, -1)
-    return SageParams(B, Hq, k.shape[1], N, d, dt, int(causal), float(sm_scale if sm_scale else 0.0),
-                      int(smooth_k), int(smooth_q), bq, bk, int(pv_accum), int(return_lse))
+    return SageParams(B, Hq, Hkv, N, d, dt, int(causal), float(sm_scale if sm_scale else 0.0),
+                      int(smooth_k), int(smooth_q), bq, bk, int(pv_accum), int(return_lse), LAYOUTS[tensor_layout])
 
 
 def workspace_bytes(p: SageParams) -> int:
@@ -160,10 +169,11 @@ def sage_attn_fwd_quantized(view: SageQuantView, o: torch.Tensor, p: SageParams,
 def sage_attn_fwd(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = None, smooth_k: bool = True,
                   smooth_q: bool = False, bq: int = 128, bk: int = 64, pv_accum: int = PV_TWO_LEVEL,
                   out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                  stream=None) -> torch.Tensor:
-    """SageAttention forward: [B,Hq,N,d] x [B,Hkv,N,d] -> [B,Hq,N,d] (input dtype)."""
+                  stream=None, tensor_layout: str = "HND") -> torch.Tensor:
+    """SageAttention forward: [B,Hq,N,d] x [B,Hkv,N,d] -> [B,Hq,N,d] (input dtype); with
+    tensor_layout "NHD" the tensors are [B,N,H,d]."""
     p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq, bk=bk,
-                    pv_accum=pv_accum)
+                    pv_accum=pv_accum, tensor_layout=tensor_layout)
     if workspace is None:
         workspace = alloc_workspace(p, q.device)
     if out is None:
@@ -176,11 +186,11 @@ def sage_attn_fwd(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = 
 def sage_attn_fwd_lse(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = None, smooth_k: bool = True,
                       smooth_q: bool = False, bq: int = 128, bk: int = 64, pv_accum: int = PV_TWO_LEVEL,
                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                      workspace: Optional[torch.Tensor] = None, stream=None):
+                      workspace: Optional[torch.Tensor] = None, stream=None, tensor_layout: str = "HND"):
     """sage_attn_fwd that also returns each row's log-sum-exp of the scores
     (fp32 [B,Hq,N], natural log, for the original keys): (out, lse)."""
     p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq, bk=bk,
-                    pv_accum=pv_accum)
+                    pv_accum=pv_accum, tensor_layout=tensor_layout)
     if workspace is None:
         workspace = alloc_workspace(p, q.device)
     if out is None:
@@ -282,9 +292,11 @@ def sage_attn_fwd_nvfp4_quantized(view: SageNvfp4View, o: torch.Tensor, p: SageP
 def sage_attn_fwd_nvfp4(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = None,
                         smooth_k: bool = True, smooth_q: bool = True, bq: int = 128,
                         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                        stream=None) -> torch.Tensor:
-    """SageAttention3-style NVFP4 forward: [B,Hq,N,128] x [B,Hkv,N,128] -> [B,Hq,N,128]."""
-    p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq)
+                        stream=None, tensor_layout: str = "HND") -> torch.Tensor:
+    """SageAttention3-style NVFP4 forward: [B,Hq,N,128] x [B,Hkv,N,128] -> [B,Hq,N,128]
+    (tensor_layout "NHD": [B,N,H,128])."""
+    p = make_params(q, k, causal=causal, sm_scale=sm_scale, smooth_k=smooth_k, smooth_q=smooth_q, bq=bq,
+                    tensor_layout=tensor_layout)
     if workspace is None:
         workspace = alloc_nvfp4_workspace(p, q.device)
     if out is None:

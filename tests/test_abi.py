@@ -47,12 +47,13 @@ def test_workspace_bytes_valid_and_invalid(L):
     assert n >= 3 * 1 * 2 * 256 * 64
     assert sage.workspace_bytes(P(smooth_q=1)) > n  # + qbar and delta_S
     for bad in (P(d=96), P(Hq=3, Hkv=2), P(N=0), P(bq=16), P(bq=256), P(bk=32), P(bk=256), P(dtype=7),
-                P(causal=2)):
+                P(causal=2), P(return_lse=2), P(layout=2)):
         assert sage.workspace_bytes(bad) == 0
     # one Q scale per 32 rows: INT8/FP8 path only (the NVFP4 smooth-Q block is 64 or 128 rows)
     assert sage.workspace_bytes(P(bq=32)) > 0
     assert sage.nvfp4_workspace_bytes(P(d=128, bq=32)) == 0
     assert sage.nvfp4_workspace_bytes(P(d=128, bq=64)) > 0
+    assert sage.workspace_bytes(P(layout=1)) == n  # NHD inputs: the same workspace
 
 
 def test_entry_points_reject_bad_arguments_on_host(L):
