@@ -39,9 +39,9 @@ FP4_PER_BF16 = 4.0  # nominal dense ratio 9 / 2.25 PFLOP/s
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch of the prefill workload: one ncu capture of attn_i8f8_kernel at B=3
-# (486.4 MB), scaled to B=4 by the number of heads.  Valid only for the kernel
+# (482.4 MB), scaled to B=4 by the number of heads.  Valid only for the kernel
 # source it was taken on (hash below); any other source reports null.
-ATTN_TRAFFIC = {"bytes": 486.4e6 * 4 / 3, "src_sha256_16": "c3a08894409178e2", "workload": "llm_prefill_causal_B4_H32_N4096_d128"}
+ATTN_TRAFFIC = {"bytes": 482.4e6 * 4 / 3, "src_sha256_16": "7059f06be6cfa67e", "workload": "llm_prefill_causal_B4_H32_N4096_d128"}
 
 
 def _attn_traffic(w: W.Workload):
