@@ -183,6 +183,7 @@ void set_out_strides(AttnArgs* a, const sage_params* p, const Dims& d) {
   a->o_bs = Hq * N * D;
   a->o_hs = p->layout == SAGE_NHD ? D : N * D;
   a->o_rs = p->layout == SAGE_NHD ? Hq * D : D;
+  a->nhd = p->layout == SAGE_NHD;
 }
 
 AttnArgs attn_args(const sage_quant_view* v, const sage_params* p, const Dims& d) {

@@ -112,7 +112,9 @@ __device__ __forceinline__ uint32_t pack2f4<__half>(float a, float b) {
 
 __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) { return make_sdesc(saddr, 128, kSwizzleNone); }
 
-template <bool CAUSAL, bool HAS_DS, typename TO>
+// NHD: o is [B, N, Hq, 128] (else [B, Hq, N, 128]); a template choice, so that
+// the register-tight epilogue computes one fixed address formula
+template <bool CAUSAL, bool HAS_DS, typename TO, bool NHD>
 __global__ void __launch_bounds__(kThreadsF4, 1)
     attn_nvfp4_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -524,8 +526,7 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
       tc_fence_after();
       const float f = s_l[i * 128 + row];
       const int64_t qrow = (int64_t)(2 * pr + i) * kTile + row;
-      // row qrow of head (b, h): one formula for either layout (strides from the host)
-      TO* out = reinterpret_cast<TO*>(a.o) + b * a.o_bs + h * a.o_hs + qrow * a.o_rs;
+      TO* out = reinterpret_cast<TO*>(a.o) + (NHD ? ((int64_t)b * a.N + qrow) * a.Hq + h : (int64_t)bh * a.N + qrow) * 128;
       const uint32_t tA = tmem + kColA + 128 * i + lane_off;
 #pragma unroll
       for (int c = 0; c < 128; c += 32) {
@@ -630,7 +631,7 @@ __global__ void __launch_bounds__(128, 1)
 template <bool CAUSAL, bool HAS_DS, typename TO>
 cudaError_t launch_nvfp4_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                            cudaStream_t st) {
-  auto k = attn_nvfp4_kernel<CAUSAL, HAS_DS, TO>;
+  auto k = a.nhd ? attn_nvfp4_kernel<CAUSAL, HAS_DS, TO, true> : attn_nvfp4_kernel<CAUSAL, HAS_DS, TO, false>;
   const int smem = (int)SmemF4::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -71,6 +71,7 @@ struct AttnArgs {
   const float* dS;  // nullptr when smooth_q is off
   void* o;          // [B,Hq,N,D] bf16/fp16 ([B,N,Hq,D] when the caller's layout is NHD)
   int64_t o_bs, o_hs, o_rs;  // element strides of o between batches, heads and rows
+  int nhd;                   // the caller's layout is NHD (NVFP4 kernel: a template choice)
   float* lse;        // [B,Hq,N] natural-log log-sum-exp of the rows' scores, or nullptr
   const float* qkm;  // [B,Hq,Np] Q_i . km (the smooth-K correction of lse / sm_scale)
   int out_fp16;
