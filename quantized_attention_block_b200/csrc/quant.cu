@@ -364,7 +364,9 @@ __device__ __forceinline__ void block_means(const T* sX, double (*s_sum)[8], flo
 // grid (Np/128, B*H), 256 threads, dynamic smem: 128 x D elements + 128
 //   SHIFT: the shift is applied (smooth_q for Q, smooth_k for K); otherwise it
 //   is identically zero and the block max runs on the raw 16-bit magnitudes.
-template <typename T, int D, int BQ, bool IS_K, bool SHIFT>
+//   QKM (Q only): also write Q_i . km per row (for the log-sum-exp); a template
+//   choice so that the plain kernel carries none of it.
+template <typename T, int D, int BQ, bool IS_K, bool SHIFT, bool QKM = false>
 __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constant__ CUtensorMap tmX, QuantArgs a) {
   constexpr int NB = kTile / BQ;
   extern __shared__ uint8_t qk_smem_raw[];
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
     }
   }
   if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh, IS_K ? a.Hkv : a.Hq)) return;
-  if (!IS_K && a.qkm != nullptr) {
+  if (!IS_K && QKM) {
     // Q_i . km of every row of the tile (fp32), from the unshifted rows: the
     // constant by which smooth K shifts row i's scores (log-sum-exp correction)
     constexpr int CH = D / 8, RG = kThreads / CH;
@@ -875,6 +877,13 @@ void (*kv_fused_kernel(const QuantArgs& a, int tiles, int smem))(CUtensorMap, CU
   return (int64_t)tiles * 2 <= (int64_t)sms * per_sm ? kf : nullptr;
 }
 
+template <typename T, int D, bool QKM>
+auto q_quant_pick(const QuantArgs& a) {
+  return a.bq == 32   ? (a.smooth_q ? qk_quant_kernel<T, D, 32, false, true, QKM> : qk_quant_kernel<T, D, 32, false, false, QKM>)
+         : a.bq == 64 ? (a.smooth_q ? qk_quant_kernel<T, D, 64, false, true, QKM> : qk_quant_kernel<T, D, 64, false, false, QKM>)
+                      : (a.smooth_q ? qk_quant_kernel<T, D, 128, false, true, QKM> : qk_quant_kernel<T, D, 128, false, false, QKM>);
+}
+
 template <typename T, int D>
 cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t st) {
   cudaError_t e;
@@ -908,9 +917,7 @@ cudaError_t launch_quant_t(const QuantArgs& a, const QuantMaps& m, cudaStream_t 
     v_quant_kernel<T, D><<<dim3(tiles, BHkv), kThreads, smem, st>>>(m.v, m.vt, a);
   }
   {
-    auto qq = a.bq == 32   ? (a.smooth_q ? qk_quant_kernel<T, D, 32, false, true> : qk_quant_kernel<T, D, 32, false, false>)
-              : a.bq == 64 ? (a.smooth_q ? qk_quant_kernel<T, D, 64, false, true> : qk_quant_kernel<T, D, 64, false, false>)
-                           : (a.smooth_q ? qk_quant_kernel<T, D, 128, false, true> : qk_quant_kernel<T, D, 128, false, false>);
+    auto qq = a.qkm ? q_quant_pick<T, D, true>(a) : q_quant_pick<T, D, false>(a);
     e = cudaFuncSetAttribute(qq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_qk);
     if (e != cudaSuccess) return e;
     qq<<<dim3(tiles, BHq), kThreads, smem_qk, st>>>(m.q, a);
