@@ -133,16 +133,17 @@ bool map_2d_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
 
 // [B*H][N][D] bf16/fp16 input as a 3D tensor (box 1 x 128 x D, no swizzle):
 // a tile that runs past N reads zeros.
-// A caller's 16-bit input as a 4D (D, N, H, B) tensor whose strides encode its
-// layout (HND: [B, H, N, D]; NHD: [B, N, H, D]); box D x 128 x 1 x 1.
+// A caller's 16-bit input as a TMA tensor: HND [B, H, N, D] as 3D (D, N, B H);
+// NHD [B, N, H, D] as 4D (D, N, H, B) with the layout in the strides.  Box
+// D x 128 (x 1 (x 1)); the quantisers pass matching coordinates.
 bool map_input(CUtensorMap* m, const void* base, uint64_t D, uint64_t N, uint64_t H, uint64_t B, int nhd) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[4] = {D, N, H, B};
+  const cuuint64_t dims[4] = {D, N, nhd ? H : B * H, B};
   const cuuint64_t strides[3] = {(nhd ? H * D : D) * 2, (nhd ? D : N * D) * 2, H * N * D * 2};
   const cuuint32_t box[4] = {(cuuint32_t)D, kTile, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, nhd ? 4 : 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

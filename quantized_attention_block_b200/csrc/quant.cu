@@ -187,11 +187,13 @@ __global__ void __launch_bounds__(kThreads) kv_stats_kernel(QuantArgs a) {
 
 // ---------------------------------------------------------------------------
 // Pass 2: one 128-row tile of Q, K or V per CTA.  The tile arrives in shared
-// memory by one TMA load (4D map (D, N, H, B); rows past N read as zeros), so
+// memory by one TMA load (3D map (D, N, B H) for HND inputs, 4D (D, N, H, B)
+// for NHD; rows past N read as zeros), so
 // the registers hold no tile and several CTAs per SM keep HBM busy; the
 // threads then sweep the tile in shared memory (block sums, block max, codes).
 template <typename T, int D>
-__device__ __forceinline__ bool load_tile(T* dst, const CUtensorMap* map, uint64_t* bar, int row0, int bh, int H) {
+__device__ __forceinline__ bool load_tile(T* dst, const CUtensorMap* map, uint64_t* bar, int row0, int bh, int H,
+                                          int nhd) {
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     mbar_fence_init();
@@ -199,7 +201,10 @@ __device__ __forceinline__ bool load_tile(T* dst, const CUtensorMap* map, uint64
   __syncthreads();
   if (threadIdx.x == 0) {
     mbar_expect_tx(bar, kTile * D * (uint32_t)sizeof(T));
-    tma_load_4d(dst, map, bar, 0, row0, bh % H, bh / H);
+    if (nhd)
+      tma_load_4d(dst, map, bar, 0, row0, bh % H, bh / H);  // (d, N, H, B) map
+    else
+      tma_load_3d(dst, map, bar, 0, row0, bh);  // (d, N, B H) map
   }
   return mbar_wait(bar, 0);
 }
@@ -388,7 +393,7 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
       for (int nb = 0; nb < NB; ++nb) s_shift[nb][c] = 0.0f;
     }
   }
-  if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh, IS_K ? a.Hkv : a.Hq)) return;
+  if (!load_tile<T, D>(sX, &tmX, &bar, (int)r0, bh, IS_K ? a.Hkv : a.Hq, a.nhd)) return;
   if (!IS_K && QKM) {
     // Q_i . km of every row of the tile (fp32), from the unshifted rows: the
     // constant by which smooth K shifts row i's scores (log-sum-exp correction)
@@ -478,7 +483,7 @@ __global__ void __launch_bounds__(kThreads)
     s_sv[c] = sv;
     if (tile == 0) a.s_v[(int64_t)bg * D + c] = sv;
   }
-  if (!load_tile<T, D>(sV, &tmX, &bar, (int)r0, bg, a.Hkv)) return;
+  if (!load_tile<T, D>(sV, &tmX, &bar, (int)r0, bg, a.Hkv, a.nhd)) return;
   v_encode<T, D>(sV, sVt, s_sv, &tmVt, tile, bg);
 }
 
@@ -552,7 +557,7 @@ __global__ void __launch_bounds__(kThreads)
   const int grp = s_item / tiles, tile = s_item % tiles;
   const int bh = grp >> 1;
   const bool is_v = (grp & 1) != 0;
-  if (!load_tile<T, D>(sX, is_v ? &tmV : &tmK, &bar, tile * kTile, bh, a.Hkv)) return;
+  if (!load_tile<T, D>(sX, is_v ? &tmV : &tmK, &bar, tile * kTile, bh, a.Hkv, a.nhd)) return;
   if (!is_v && !SMOOTH_K) {  // km = 0: nothing to wait for
     if (tile == 0 && threadIdx.x < D) a.km[(int64_t)bh * D + threadIdx.x] = 0.0f;
     qk_encode<T, D, BK, true, false>(sX, s_shift, s_red, s_bmax, bh, tile, a);

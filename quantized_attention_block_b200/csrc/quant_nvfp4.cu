@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads) q_quant_nvfp4_kernel(const __grid_co
   __shared__ uint64_t bar;
   const int bh = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
-  if (!load_tile<T, D>(sX, &tmQ, &bar, (int)r0, bh, a.Hq)) return;
+  if (!load_tile<T, D>(sX, &tmQ, &bar, (int)r0, bh, a.Hq, a.nhd)) return;
   if (SHIFT) block_means<T, D, BQ>(sX, s_sum, s_mean, bh, tile, a);
   __syncthreads();
   nvfp4_encode_tile<T, BQ>(sX, SHIFT ? s_mean : nullptr, s_sf, rows_valid(a.N, r0, kTile),
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kThreads) k_fused_nvfp4_kernel(const __grid_co
   if (threadIdx.x == 0) s_item = atomicAdd(a.kv_sync, 1);
   __syncthreads();
   const int bg = s_item / tiles, tile = s_item % tiles;
-  if (!load_tile<T, D>(sX, &tmK, &bar, tile * kTile, bg, a.Hkv)) return;
+  if (!load_tile<T, D>(sX, &tmK, &bar, tile * kTile, bg, a.Hkv, a.nhd)) return;
   if constexpr (SMOOTH_K) {
     const int ch = threadIdx.x % CH, rg = threadIdx.x / CH, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     double cs[8];
