@@ -214,39 +214,32 @@ __global__ void __launch_bounds__(kThreads) k_fused_nvfp4_kernel(const __grid_co
 
 // ---------------------------------------------------------------------------
 // V: NVFP4 along tokens (16-token groups per channel), transposed to
-// [D][Np/2].  The tile is staged in shared memory; each thread encodes one
-// (channel, 16-token group) at a time, consecutive threads taking consecutive
-// channels; codes go through shared memory so the global stores are 16-byte
-// rows.  grid (Np/128, B*Hkv), 256 threads.
+// [D][Np/2].  The tile arrives in shared memory by one TMA load; each thread
+// encodes (channel, 16-token group) items, consecutive threads taking
+// consecutive channels, and keeps the codes in registers; after a barrier they
+// are written over the consumed tile so that the global stores are 16-byte
+// rows.  grid (Np/128, B*Hkv), 256 threads, dynamic smem 128 x 128 elements + 128.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) v_quant_nvfp4_kernel(QuantArgs a) {
-  constexpr int D = kF4D, CH = D / 8, RG = kThreads / CH, NP = kTile / RG, kPitch = D + 8;
-  __shared__ __align__(16) T sV[kTile * kPitch];
-  __shared__ __align__(16) uint8_t sVt[D * (kTile / 2)];
+__global__ void __launch_bounds__(kThreads) v_quant_nvfp4_kernel(const __grid_constant__ CUtensorMap tmV, QuantArgs a) {
+  constexpr int D = kF4D, IT = (D * 8) / kThreads;  // (channel, group) items per thread
+  extern __shared__ uint8_t v4_smem_raw[];
+  T* sV = reinterpret_cast<T*>(align128(v4_smem_raw));
+  uint8_t* sVt = reinterpret_cast<uint8_t*>(sV);  // [D][64] code bytes, over the consumed tile
   __shared__ __align__(16) uint8_t s_sf[1024];
+  __shared__ uint64_t bar;
   const int bg = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
-  const int valid = rows_valid(a.N, r0, kTile);
-  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
-  const T* V = reinterpret_cast<const T*>(a.v) + row_offset(bg, 0, a.Hkv, a.N, D, a.nhd);
-  const int64_t rs = row_stride(a.Hkv, D, a.nhd);
+  if (!load_tile<T, D>(sV, &tmV, &bar, (int)r0, bg, a.Hkv, a.nhd)) return;  // rows past N are zero
+  uint2 codes[IT];
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int r = rg + p * RG;
-    uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (r < valid) u = __ldg(reinterpret_cast<const uint4*>(V + (r0 + r) * rs + ch * 8));
-    *reinterpret_cast<uint4*>(sV + r * kPitch + ch * 8) = u;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int it = 0; it < (D * 8) / kThreads; ++it) {
+  for (int it = 0; it < IT; ++it) {
     const int item = threadIdx.x + it * kThreads;
     const int c = item % D, grp = item / D;
     float x[16];
     float am = 0.0f;
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
-      x[u] = to_float(sV[(grp * 16 + u) * kPitch + c]);
+      x[u] = to_float(sV[(grp * 16 + u) * D + c]);
       am = fmaxf(am, fabsf(x[u]));
     }
     const uint32_t sc = cvt_e4m3(__fdiv_rn(am, 6.0f));
@@ -258,9 +251,15 @@ __global__ void __launch_bounds__(kThreads) v_quant_nvfp4_kernel(QuantArgs a) {
       hi[u] = x[8 + u];
     }
     const float rd = sd == 0.0f ? 0.0f : __frcp_rn(sd);
-    const uint2 codes = sd == 0.0f ? make_uint2(0u, 0u) : make_uint2(quant_e2m1x8(lo, sd, rd), quant_e2m1x8(hi, sd, rd));
-    *reinterpret_cast<uint2*>(sVt + c * (kTile / 2) + grp * 8) = codes;
+    codes[it] = sd == 0.0f ? make_uint2(0u, 0u) : make_uint2(quant_e2m1x8(lo, sd, rd), quant_e2m1x8(hi, sd, rd));
     s_sf[sf_byte(c, grp)] = (uint8_t)sc;
+  }
+  __syncthreads();  // every thread has read the tile
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int item = threadIdx.x + it * kThreads;
+    const int c = item % D, grp = item / D;
+    *reinterpret_cast<uint2*>(sVt + c * (kTile / 2) + grp * 8) = codes[it];
   }
   __syncthreads();
   uint8_t* v4t = a.v4t + (int64_t)bg * D * (a.Np / 2) + r0 / 2;
@@ -320,7 +319,9 @@ cudaError_t launch_quant_nvfp4_t(const QuantArgs& a, const QuantMaps& m, cudaStr
     kv_stats_kernel<T, kF4D><<<dim3((a.N + kStatRows - 1) / kStatRows, BHkv), kThreads, 0, st>>>(s);
     k_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, 0, st>>>(s);
   }
-  v_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, 0, st>>>(s);
+  e = cudaFuncSetAttribute(v_quant_nvfp4_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  v_quant_nvfp4_kernel<T><<<dim3(tiles, BHkv), kThreads, smem, st>>>(m.v, s);
   {
     auto qq = a.bq == 64 ? (a.smooth_q ? q_quant_nvfp4_kernel<T, 64, true> : q_quant_nvfp4_kernel<T, 64, false>)
                          : (a.smooth_q ? q_quant_nvfp4_kernel<T, 128, true> : q_quant_nvfp4_kernel<T, 128, false>);
