@@ -16,7 +16,9 @@
  *     of K, broadcast to the Q heads of a KV group.
  *
  * Conventions for every entry point:
- *   - Tensors are HND: [B, H, N, d], contiguous, d fastest.
+ *   - Tensors are HND [B, H, N, d] (default) or NHD [B, N, H, d] (p->layout),
+ *     contiguous, d fastest.  Quantised tensors in the workspace, qkm and lse
+ *     are head-major in either case.
  *   - Every pointer argument is a DEVICE pointer owned by the caller unless
  *     stated otherwise; the library never allocates device memory.  Scratch
  *     lives in a caller-provided workspace of sage_workspace_bytes() bytes.
@@ -123,7 +125,7 @@ SAGE_API size_t sage_workspace_bytes(const sage_params *p);
  *   s_q/s_k = amax_block |x| / 127,  code = clamp(rint(x / s), -127, 127)
  *   s_v[c]  = amax_n |V[n,c]| / 448, v8t   = E4M3_rn_satfinite(V / s_v)
  *   dS[i,j] = qbar_i . gamma(K_j)            (smooth_q only; fp32 accumulation)
- * q, k, v: device [B,H,N,d] in p->dtype.  Fills *view (host struct) with
+ * q, k, v: device [B,H,N,d] (or [B,N,H,d], p->layout) in p->dtype.  Fills *view (host struct) with
  * pointers into `workspace`.  Quantised tensors and scales are bit-exact with
  * the plain definitions above.
  * For d = 128, K and V are read from HBM once when the ceil(N/128) tiles of
