@@ -326,6 +326,77 @@ def test_nvfp4_two_level_p_hand_worked():
     assert abs(out[0, 0] - expect) < 1e-6
 
 
+def test_e4m3_p_path_hand_worked_4x4_causal_growing_max():
+    """Hand-worked 4x4 causal case, K tile = 2 keys, so the online softmax of rows
+    2 and 3 spans two tiles and their max grows in the second one.
+    d = 1; s_q = s_k = 1, sm_scale = 1, so S[r, c] = Q^[r] K^[c].
+    Q^ = [1, 1, 1, 2], K^ = [-1, -2, 0, -3], V = [1, 2, 0.5, 4], s_v = 0.25.
+      row 0: key 0: S = [-1]; P~ = [1]; l = 1; P^ = [448]; O = 448
+             out = 448 / 1 / 448 * 0.25 = 0.25
+      row 1: keys 0, 1: S = [-1, -2], m = -1; P~ = [1, e^-1], l = 1 + e^-1;
+             448 e^-1 = 164.8 -> E4M3 160 (grid step 16 in [128, 256));
+             O = 448 * 1 + 160 * 2 = 768
+      row 2: tile 0 as row 1 (m = -1, l0 = 1 + e^-1, O0 = 768); tile 1 holds
+             key 2 only (key 3 is causally masked): S = [0], m grows -1 -> 0,
+             alpha = e^-1; P~ = [1] -> 448; O_t = 448 * 0.5 = 224
+             l = e^-1 l0 + 1, O = e^-1 * 768 + 224
+      row 3: tile 0: S = [-2, -4], m = -2; P~ = [1, e^-2]; 448 e^-2 = 60.63 ->
+             E4M3 60 (step 4 in [32, 64)); O0 = 448 + 60 * 2 = 568, l0 = 1 + e^-2
+             tile 1: S = [0, -6], m grows -2 -> 0, alpha = e^-2;
+             P~ = [1, e^-6]; 448 e^-6 = 1.1105 -> E4M3 1.125 (step 1/8 in
+             [1, 2)); O_t = 448 * 0.5 + 1.125 * 4 = 228.5
+             l = e^-2 l0 + 1 + e^-6, O = e^-2 * 568 + 228.5
+    out = O / l / 448 * 0.25 in every row."""
+    Qv = np.array([[1.0], [1.0], [1.0], [2.0]])
+    Kv = np.array([[-1.0], [-2.0], [0.0], [-3.0]])
+    Vv = np.array([[1.0], [2.0], [0.5], [4.0]])
+    one = np.ones(4)
+    out = oracle._attn_core(Qv, Kv, Vv, one, one, None, 64, np.array([0.25]), 4, 1, True, 1.0, 1, 1, 0, 4,
+                            tile=2)
+    e = math.exp
+    l2 = e(-1) * (1 + e(-1)) + 1
+    l3 = e(-2) * (1 + e(-2)) + 1 + e(-6)
+    expect = np.array([
+        448.0 / 1.0,
+        768.0 / (1 + e(-1)),
+        (e(-1) * 768.0 + 224.0) / l2,
+        (e(-2) * 568.0 + 228.5) / l3,
+    ]) / 448.0 * 0.25
+    np.testing.assert_allclose(out[:, 0], expect, rtol=2e-6)
+
+
+def test_nvfp4_two_level_p_per_16_groups_hand_worked():
+    """SA3 two-level P quantisation of one 64-key tile whose four 16-key groups
+    have different maxima, so one s_P2 per 16 keys, per 32 or per tile give
+    different outputs.  d = 1, Q = 1, sm_scale = 1, so S = K; the row max is key 0
+    (S = 0), hence P~ = e^S and s_P1 = 1 / 2688, P2 = 2688 P~.
+      group 0: P~ = [1, 15 x e^-30]: amax 2688 -> s_P2 = E4M3(448) = 448;
+               P2 / s_P2 = [6, ~0] -> E2M1 [6, 0]: P^ s_P2 s_P1 = [1, 0...]
+      group 1: 16 x P~ = 0.1: P2 = 268.8, s_P2 = E4M3(44.8) = 44 (step 4 in
+               [32, 64)); 268.8 / 44 = 6.11 -> 6: each 6 * 44 / 2688 = 264 / 2688
+      group 2: P~ = [0.25, 15 x 0.05]: P2 = [672, 134.4], s_P2 = E4M3(112) = 112;
+               [6, 1.2] -> E2M1 [6, 1]: [0.25, 15 x 112 / 2688]
+      group 3: 16 x P~ = 0.02: P2 = 53.76, s_P2 = E4M3(8.96) = 9;
+               5.97 -> E2M1 6: each 54 / 2688
+    V = 1, 2, 4, 8 on groups 0..3; l = 1 + 1.6 + 1 + 0.32 = 3.92 (fp32 P~, before
+    quantisation).  One s_P2 per 32 keys gives 0.9035 (V = 1) instead of
+    0.9612; one per tile gives 0.9779."""
+    K = np.concatenate([[0.0], np.full(15, -30.0), np.full(16, math.log(0.1)), [math.log(0.25)],
+                        np.full(15, math.log(0.05)), np.full(16, math.log(0.02))])[:, None]
+    Q = np.ones((64, 1))
+    V = np.repeat([1.0, 2.0, 4.0, 8.0], 16)[:, None]
+    g = np.array([1.0,
+                  16 * 264 / 2688,
+                  0.25 + 15 * 112 / 2688,
+                  16 * 54 / 2688])
+    l = 1 + 16 * 0.1 + 0.25 + 15 * 0.05 + 16 * 0.02
+    out = oracle._attn_core(Q, K, V, None, None, None, 64, None, 64, 1, False, 1.0, 2, 1, 0, 1, tile=64)
+    assert abs(out[0, 0] - (g @ np.array([1.0, 2.0, 4.0, 8.0])) / l) < 2e-6 * out[0, 0]
+    ones = np.ones((64, 1))
+    out1 = oracle._attn_core(Q, K, ones, None, None, None, 64, None, 64, 1, False, 1.0, 2, 1, 0, 1, tile=64)
+    assert abs(out1[0, 0] - g.sum() / l) < 2e-6
+
+
 def test_oracle_int8_fp8_cosine_vs_exact_small_workloads():
     """Whole oracle vs fp64 exact: cosine >= 0.998 on each INT8/FP8 recipe at a
     size of a few tiles with a ragged tail (full-size versions run on the GPU machine)."""
