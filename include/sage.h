@@ -218,11 +218,16 @@ SAGE_API sage_status sage_debug_bounded_wait(uint32_t timeout_us, void *stream);
  *   - q, k, v, o: device pointers as for sage_attn_fwd (caller-owned).
  *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library
  *     routine.
- *   - Returns SAGE_ERR_WORKSPACE_TOO_SMALL when sage_workspace_bytes(p)
- *     exceeds SAGE_STATIC_SCRATCH_BYTES (nothing is enqueued then).
+ *   - Parameters are checked first, with the statuses sage_attn_fwd gives
+ *     (e.g. SAGE_ERR_UNSUPPORTED_HEADDIM); then SAGE_ERR_WORKSPACE_TOO_SMALL
+ *     when sage_workspace_bytes(p) exceeds SAGE_STATIC_SCRATCH_BYTES; then
+ *     SAGE_ERR_UNSUPPORTED_ARCH off sm_100.  Nothing is enqueued on an error.
  *   - The first call on a device looks up the array's device address on
- *     that device (the device must be current) and caches it; make that first
- *     call before any stream capture.
+ *     that device (the device must be current) and caches it with the id of
+ *     the device's context; make that first call before any stream capture.
+ *     A context re-created on that device (after cudaDeviceReset) is noticed
+ *     by its new id and the address is looked up again, so again make that
+ *     next call outside a capture.
  *   - All calls on a device share the one array, and it keeps whatever the
  *     last call left in it.  Calls whose work overlaps on the GPU (different
  *     streams, or host threads without ordering) race on it; order them.
@@ -309,12 +314,32 @@ SAGE_API sage_status sage_debug_qk_nvfp4(const sage_nvfp4_view *view, const sage
                                          void *stream);
 
 /*
- * Accuracy probe of the FMA-pipe exponential the attention kernel uses for part
- * of each row of P (so that not every exp2 waits for the MUFU): y[i] = 2^x[i]
- * for n device floats, computed by the same device function.  Valid for
- * -126 <= x <= 100; x < -126 gives 2^-126 or less (the kernel's masked scores).
+ * Accuracy probe of the FMA-pipe exponential (a Cody-Waite range reduction and
+ * a degree-4 polynomial on the FMA and ALU pipes, so that an exp2 need not use
+ * the MUFU): y[i] = 2^x[i] for n device floats, computed by the same device
+ * function the attention kernels can use for a share of their exponentials
+ * (a compile-time choice; the shipped kernels compute every exponential of P
+ * on the MUFU, which measured faster).  Valid for -126 <= x <= 100; x < -126
+ * gives 2^-126 or less (the kernel's masked scores).
  */
 SAGE_API sage_status sage_debug_exp2_poly(const float *x, float *y, int32_t n, void *stream);
+
+/*
+ * Tensor-core rate probe (the measured peak that the attention kernels are
+ * compared with; the pages give no counterpart for B200).  Launches `ctas`
+ * CTAs (0: one per SM), each issuing `iters` back-to-back passes of
+ * tcgen05.mma with M = 128 on operand tiles resident in shared memory,
+ * accumulating in TMEM:
+ *   kind 0: kind::i8 (s8, s32 accumulator), n = 64, 128 or 256, 4 x K = 32 per pass
+ *   kind 1: kind::f8f6f4 (E4M3, f32 accumulator), n = 64, 128 or 256, 4 x K = 32
+ *   kind 2: kind::mxf4nvf4 block16 (E2M1 with UE4M3 scales), n = 128, 2 x K = 64
+ * *ops (host) receives the launch's operation count, 2 x 128 x n x 128 per
+ * pass per CTA; dividing it by the launch's duration (CUDA events on
+ * `stream`) gives the rate.  1 <= iters <= 2,000,000.  SAGE_ERR_INVALID_ARG
+ * for an unsupported (kind, n).
+ */
+SAGE_API sage_status sage_debug_mma_rate(int32_t kind, int32_t n, int32_t iters, int32_t ctas, double *ops,
+                                         void *stream);
 
 /*
  * Number of kernels sage_quant_qkv enqueues for p on the current device (not

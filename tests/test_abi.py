@@ -72,3 +72,25 @@ def test_entry_points_reject_bad_arguments_on_host(L):
     st = L.sage_debug_qk_int32(None, ctypes.byref(p), 0, 0, 0, 0, None, None)
     assert st == 1
     assert L.sage_status_string(7) == b"SAGE_ERR_TIMEOUT"
+
+
+def test_noalloc_reports_parameter_errors_like_sage_attn_fwd(L):
+    """The no-allocation entry point validates the parameters before it looks at
+    the static scratch size, so unsupported parameters get the same status as
+    from sage_attn_fwd (checked on the host, no CUDA call is reached)."""
+    for bad, want in ((P(d=96), 2), (P(dtype=3), 3), (P(Hq=3, Hkv=2), 1), (P(N=0), 1)):
+        st_ws = L.sage_attn_fwd(None, None, None, None, ctypes.byref(bad), None, 0, None)
+        st_na = L.sage_attn_fwd_noalloc(None, None, None, None, ctypes.byref(bad), None)
+        assert st_na == st_ws == want, (bad.d, bad.dtype, st_na, st_ws)
+    assert L.sage_attn_fwd_noalloc(None, None, None, None, None, None) == 1
+    # far beyond the 32 MiB static scratch: rejected before any device query
+    big = P(B=4, Hq=32, Hkv=32, N=4096, d=128)
+    assert L.sage_attn_fwd_noalloc(None, None, None, None, ctypes.byref(big), None) == 5
+
+
+def test_mma_rate_probe_rejects_bad_shapes_on_host(L):
+    ops = ctypes.c_double(0.0)
+    for kind, n, iters in ((3, 128, 10), (0, 96, 10), (2, 256, 10), (1, 128, 0), (1, 128, 3_000_000)):
+        assert L.sage_debug_mma_rate(kind, n, iters, 0, ctypes.byref(ops), None) == 1, (kind, n, iters)
+    assert L.sage_debug_mma_rate(0, 128, 10, 0, None, None) == 1
+
