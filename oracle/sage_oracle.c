@@ -23,7 +23,7 @@
  *          analysis), sections "Online Softmax" (m, l, rescale update) and
  *          "精度与量化策略" (per-block INT8, per-channel FP8 V, smooth_k).
  *
- * Readings taken where the pages are silent (each one is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - means are summed in fp64 and rounded once to fp32;
  *   - INT8 scale = amax / 127 (fp32 division), code = clamp(rint(x / scale)),
  *     x / scale an IEEE fp32 division, rint = round-half-to-even;

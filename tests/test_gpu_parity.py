@@ -269,9 +269,11 @@ def test_fp8_accumulator_precision_probe():
 
 
 def test_fma_pipe_exp2_accuracy():
-    """The polynomial exp2 the softmax uses for part of each row: relative error
-    against fp64 exp2 below 1.2e-5 over the range the kernel feeds it (scores
-    minus the row max plus log2 448), exact zero-ish for masked scores."""
+    """The FMA-pipe polynomial exp2 the softmax can take for a share of its
+    exponentials (a compile-time option; the shipped kernels use the MUFU for
+    all of them): relative error against fp64 exp2 below 1.2e-5 over the range
+    the kernel would feed it (scores minus the row max plus log2 448), and a
+    tiny non-negative value for masked scores."""
     x = torch.cat([torch.linspace(-125.0, 9.0, 2_000_001), torch.tensor([0.0, 1.0, -1.0, 8.807354922057604])])
     y = sage.sage_debug_exp2_poly(x.cuda()).cpu().double()
     ref = torch.exp2(x.double())
@@ -279,3 +281,22 @@ def test_fma_pipe_exp2_accuracy():
     assert rel < 1.2e-5, rel
     masked = sage.sage_debug_exp2_poly(torch.tensor([-float("inf"), -1e30, -500.0]).cuda()).cpu()
     assert torch.all(masked >= 0) and torch.all(masked <= 2.0 ** -125)
+
+
+def test_mma_rate_probe_runs_every_shape():
+    """The tensor-core rate probe bench.py divides by: every (kind, N) launches,
+    counts 2 M N K per instruction, and lands in a plausible range for one B200
+    (hundreds to a few thousand dense TOPS)."""
+    st = torch.cuda.current_stream()
+    for kind, n in (("i8", 256), ("i8", 128), ("i8", 64), ("f8", 256), ("f8", 128), ("f8", 64), ("f4", 128)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        ops = sage.sage_debug_mma_rate(kind, n, 20000, 0, st)
+        e1.record(st)
+        torch.cuda.synchronize()
+        assert sage.sage_last_device_error() == 0
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        assert ops == 2.0 * 128 * n * 128 * 20000 * sms
+        tops = ops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        assert 100.0 < tops < 20000.0, (kind, n, tops)
+
