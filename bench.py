@@ -70,9 +70,34 @@ def _dist():
     return ws, rank, local
 
 
+_SAMPLER_CODE = r"""
+import sys, time
+import pynvml as nv
+nv.nvmlInit()
+try:
+    h = nv.nvmlDeviceGetHandleByPciBusId(sys.argv[1])
+except Exception:
+    h = nv.nvmlDeviceGetHandleByIndex(int(sys.argv[3]))
+period = float(sys.argv[2])
+print("max", nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM), flush=True)
+while True:
+    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+    try:
+        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+    except Exception:
+        rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+    print(time.monotonic_ns(), sm, rs, pw, flush=True)
+    time.sleep(period)
+"""
+
+
 class ClockSampler:
     """Samples SM clock, power and clock-event (throttle) reasons through NVML
-    every few milliseconds while the timed region runs."""
+    every few milliseconds from a separate process (its own interpreter, so the
+    launching thread cannot starve it), time-stamped with the system monotonic
+    clock.  mark() brackets a region; summary() reports the samples inside the
+    marked regions."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
@@ -81,66 +106,60 @@ class ClockSampler:
         self.dev = torch_device
         self.period = period_s
         self.samples = []
+        self.regions = {}
         self.err = None
-        self._stop = None
+        self.proc = None
+        self.max_sm = None
 
     def __enter__(self):
-        import threading
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            # match the torch device to an NVML device by PCI domain/bus/device numbers
             props = torch.cuda.get_device_properties(self.dev)
-            self.h = None
-            for idx in range(pynvml.nvmlDeviceGetCount()):
-                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
-                info = pynvml.nvmlDeviceGetPciInfo(h)
-                if (int(info.bus), int(info.device), int(info.domain)) == (
-                        int(getattr(props, "pci_bus_id", -1)), int(getattr(props, "pci_device_id", -1)),
-                        int(getattr(props, "pci_domain_id", -1))):
-                    self.h = h
-                    break
-            if self.h is None:
-                self.h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
-            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.nv = pynvml
+            bus = "%08X:%02X:%02X.0" % (int(props.pci_domain_id), int(props.pci_bus_id), int(props.pci_device_id))
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_CODE, bus, str(self.period), str(self.dev)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+            first = self.proc.stdout.readline().split()
+            if len(first) != 2 or first[0] != "max":
+                raise RuntimeError("sampler did not start: " + self.proc.stderr.read()[-300:])
+            self.max_sm = int(first[1])
         except Exception as e:  # pragma: no cover
             self.err = f"nvml unavailable: {e}"
-            return self
-        self._stop = threading.Event()
-
-        def run():
-            nv = self.nv
-            while not self._stop.is_set():
-                try:
-                    sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
-                    try:
-                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                    except Exception:
-                        rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-                    pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
-                    self.samples.append((sm, rs, pw))
-                except Exception as e:  # pragma: no cover
-                    self.err = str(e)
-                self._stop.wait(self.period)
-
-        self.t = threading.Thread(target=run, daemon=True)
-        self.t.start()
+            self.proc = None
         return self
 
-    def __exit__(self, *exc):
-        if self._stop is not None:
-            self._stop.set()
-            self.t.join(timeout=2)
+    def mark(self, name: str, begin: bool):
+        t = time.monotonic_ns()
+        if begin:
+            self.regions[name] = [t, None]
+        else:
+            self.regions[name][1] = t
 
-    def summary(self):
-        if not self.samples:
+    def __exit__(self, *exc):
+        if self.proc is None:
+            return
+        time.sleep(3 * self.period)
+        self.proc.kill()
+        out, _ = self.proc.communicate(timeout=5)
+        for ln in out.splitlines():
+            f = ln.split()
+            if len(f) == 4:
+                self.samples.append((int(f[0]), int(f[1]), int(f[2]), float(f[3])))
+
+    def summary(self, region: str = "timed"):
+        if self.proc is None and not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"]}
-        sm = [x[0] for x in self.samples]
-        reasons = sorted({name for _, rs, _ in self.samples for bit, name in self.REASONS.items() if rs & bit})
+        t0, t1 = self.regions.get(region, [0, 1 << 62])
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not inside:
+            # no sample landed in a very short region: the one just before it
+            before = [x for x in self.samples if x[0] < t0]
+            inside = before[-1:]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_sm, "reasons": ["no samples"]}
+        sm = [x[1] for x in inside]
+        reasons = sorted({name for _, _, rs, _ in inside for bit, name in self.REASONS.items() if rs & bit})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_sm, "sm_min_mhz": min(sm),
-                "reasons": reasons, "samples": len(self.samples),
-                "power_w_max": max(x[2] for x in self.samples), "source": "nvml"}
+                "reasons": reasons, "samples": len(inside), "region_ms": (t1 - t0) / 1e6,
+                "power_w_max": max(x[3] for x in inside), "source": "nvml (separate process, 2 ms period)"}
 
 
 def _barrier(ws):
@@ -213,11 +232,13 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
     with ClockSampler(torch.cuda.current_device()) as clk:
         _barrier(ws)
         torch.cuda.synchronize()
+        clk.mark("timed", True)
         t0.record(stream)
         for i in range(steps):
             step(attn_ev[i])
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.mark("timed", False)
         _barrier(ws)
     ms_total = t0.elapsed_time(t1)
     ms_attn = sum(a.elapsed_time(b) for a, b in attn_ev) / steps
@@ -306,6 +327,42 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
     return res
 
 
+# (kind, N) shapes of the tensor-core rate probe: M = 128 throughout; the
+# attention kernels use i8 N = 128 (Q K^T), f8 N = d (P V) and f4 N = 128
+MMA_SHAPES = (("i8", 256), ("i8", 128), ("i8", 64), ("f8", 256), ("f8", 128), ("f8", 64), ("f4", 128))
+
+
+def measure_mma_peaks(target_ms: float = 30.0):
+    """Measured tensor-core peaks of this GPU at the clocks of this run: the
+    library's rate probe (one CTA per SM, back-to-back tcgen05.mma on resident
+    shared-memory tiles) per kind and N, timed with CUDA events on the
+    launching stream; each launch is sized to about target_ms."""
+    from quantized_attention_block_b200 import sage
+
+    stream = torch.cuda.current_stream()
+    rates = {}
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        clk.mark("timed", True)
+        for kind, n in MMA_SHAPES:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            iters = 2000
+            for _ in range(2):  # calibrate the length, then measure
+                e0.record(stream)
+                ops = sage.sage_debug_mma_rate(kind, n, iters, 0, stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1)
+                tops = ops / (ms * 1e-3) / 1e12
+                iters = int(min(2_000_000, max(2000, iters * target_ms / max(ms, 1e-3))))
+            rates[f"{kind}_n{n}"] = tops
+        clk.mark("timed", False)
+    assert sage.sage_last_device_error() == 0
+    best = {k: max(v for key, v in rates.items() if key.startswith(k + "_")) for k in ("i8", "f8", "f4")}
+    return {"tops": rates, "best": best, "clocks": clk.summary(),
+            "how": "sage_debug_mma_rate: 1 CTA per SM, tcgen05.mma M=128 back to back on resident smem tiles, "
+                   "CUDA events, ~%.0f ms per launch" % target_ms}
+
+
 def oracle_sample(w: W.Workload, heads: int, tiles: int, threads: int, batches: int = 1):
     """Time the CPU oracle on a bounded sample: quantise `batches` x `heads`
     (b, h) pairs and run the attention of the last `tiles` Q tiles of each (the
@@ -351,6 +408,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--override", default="", help="workload fields, e.g. B=1,Hq=16,Hkv=16 (profiling cases)")
     ap.add_argument("--pv-accum", choices=["auto", "two_level", "tmem_fp32"], default="auto")
+    ap.add_argument("--no-mma-peaks", action="store_true",
+                    help="skip the tensor-core rate probe (the roofline then uses bf16 burst x nominal ratio)")
     args = ap.parse_args()
 
     ws, rank, local = _dist()
@@ -395,7 +454,6 @@ def main():
         torch.cuda.set_device(0)
 
     peaks, peak_kind = _peaks()
-    peak_tops = peaks["bf16_tflops_sustained"] * INT8_FP8_PER_BF16
     mode = pv_mode(w, args.pv_accum)
     config["pv_accum"] = ["two_level", "tmem_fp32"][mode]
     res = run_sage(w, args.steps, args.warmup, ws, rank, local, not args.no_e2e, mode,
@@ -403,21 +461,41 @@ def main():
     ops = w.ops()
     value = weak_scaling_tops(ops, res["ms_step"], ws)
     attn_tops = ops / (res["ms_attn"] * 1e-3) / 1e12
+    # roofline denominators: the tensor-core peaks measured in this run (the
+    # INT8/FP8 kernel does equal Q K^T (i8) and P V (f8) work, so its peak is
+    # the harmonic mean of the two rates); without the probe, bf16 burst x the
+    # nominal dense ratio
+    mma = None if args.no_mma_peaks else measure_mma_peaks()
+    if mma is not None:
+        b = mma["best"]
+        peak_i8f8 = 2.0 / (1.0 / b["i8"] + 1.0 / b["f8"])
+        peak_f4 = b["f4"]
+        peak_src = (f"measured in this run (sage_debug_mma_rate): i8 {b['i8']:.0f}, f8 {b['f8']:.0f} TOPS "
+                    f"(best N), harmonic mean for equal QK^T / PV work")
+        peak_src_f4 = f"measured in this run (sage_debug_mma_rate): f4 {b['f4']:.0f} TOPS"
+    else:
+        peak_i8f8 = peaks["bf16_tflops"] * INT8_FP8_PER_BF16
+        peak_f4 = peaks["bf16_tflops"] * FP4_PER_BF16
+        peak_src = (f"{peak_kind}: bf16 burst {peaks['bf16_tflops']} x {INT8_FP8_PER_BF16} "
+                    f"(nominal int8/fp8 : bf16)")
+        peak_src_f4 = f"{peak_kind}: bf16 burst {peaks['bf16_tflops']} x {FP4_PER_BF16} (nominal fp4 : bf16)"
+    peak_tops = peak_i8f8
     extra = {}
     for name in [x for x in args.extra_workloads.split(",") if x and x != "none"]:
         we = W.get(name)
         me = pv_mode(we, args.pv_accum)
         r = run_sage(we, max(3, args.steps // 4), 3, ws, rank, local, False, me, time_other_mode=True)
-        pk = peaks["bf16_tflops_sustained"] * (FP4_PER_BF16 if we.nvfp4 else INT8_FP8_PER_BF16)
+        pk = peak_f4 if we.nvfp4 else peak_i8f8
         extra[we.name] = {"pv_accum": "scaled_tmem_fp32" if we.nvfp4 else ["two_level", "tmem_fp32"][me],
                           "path": "nvfp4" if we.nvfp4 else "int8_fp8",
                           "step_tops": we.ops() / (r["ms_step"] * 1e-3) / 1e12,
                           "attn_kernel_tops": we.ops() / (r["ms_attn"] * 1e-3) / 1e12,
                           "ms_step": r["ms_step"], "ms_attn": r["ms_attn"],
                           "attn_frac_of_peak": we.ops() / (r["ms_attn"] * 1e-3) / 1e12 / pk,
-                          "peak_tops": pk}
+                          "peak_tops": pk, "clocks": r["clocks"]}
         if "ms_attn_other_mode" in r:
             extra[we.name]["attn_kernel_tops_other_mode"] = we.ops() / (r["ms_attn_other_mode"] * 1e-3) / 1e12
+            extra[we.name]["attn_frac_of_peak_other_mode"] = extra[we.name]["attn_kernel_tops_other_mode"] / pk
     line = {
         "metric": metric, "value": value, "unit": "TOPS", "n_gpus": ws, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": res["ms_step"], "higher_is_better": True,
@@ -429,11 +507,13 @@ def main():
                                             if "ms_attn_other_mode" in res else None),
         "roofline": {"bound": "tensor", "kernel": "attn_i8f8_kernel", "achieved": attn_tops,
                      "peak": peak_tops, "unit": "TFLOP/s", "frac": attn_tops / peak_tops,
-                     "peak_source": f"{peak_kind}: bf16 sustained {peaks['bf16_tflops_sustained']} x "
-                                    f"{INT8_FP8_PER_BF16} (nominal int8/fp8 : bf16)",
+                     "peak_source": peak_src, "peak_source_fp4": peak_src_f4,
+                     "peak_bf16_burst_x_ratio": peaks["bf16_tflops"] * INT8_FP8_PER_BF16,
                      "traffic": _attn_traffic(w), "traffic_unit": "bytes per launch"},
         "clocks": res["clocks"], "gpu_launches": res["gpu_launches"], "workloads": extra,
     }
+    if mma is not None:
+        line["tensor_peaks_measured"] = mma
     if "e2e" in res:
         e = res["e2e"]
         line["e2e"] = {"value": weak_scaling_tops(ops, e["ms_step"], ws), "unit": "TOPS",

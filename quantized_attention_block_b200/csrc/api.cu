@@ -637,6 +637,21 @@ sage_status sage_debug_f8_accum_probe(float* out8, void* stream) {
   return from_cuda(launch_f8_accum_probe(out8, static_cast<cudaStream_t>(stream)));
 }
 
+sage_status sage_debug_mma_rate(int32_t kind, int32_t n, int32_t iters, int32_t ctas, double* ops, void* stream) {
+  if (!ops || iters < 1 || iters > 2000000 || ctas < 0 || ctas > 4096) return SAGE_ERR_INVALID_ARG;
+  if (mma_rate_ops(kind, n, 1, 1) == 0.0) return SAGE_ERR_INVALID_ARG;
+  sage_status s = check_arch();
+  if (s != SAGE_OK) return s;
+  if (ctas == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+  }
+  *ops = mma_rate_ops(kind, n, iters, ctas);
+  return from_cuda(launch_mma_rate(kind, n, iters, ctas, static_cast<cudaStream_t>(stream)));
+}
+
 const char* sage_status_string(sage_status s) {
   switch (s) {
     case SAGE_OK: return "SAGE_OK";

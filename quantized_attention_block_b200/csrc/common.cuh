@@ -104,6 +104,9 @@ cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUt
 cudaError_t launch_bounded_wait_probe(cudaStream_t st);
 cudaError_t launch_exp2_poly_probe(const float* x, float* y, int n, cudaStream_t st);
 cudaError_t launch_f8_accum_probe(float* out, cudaStream_t st);
+// tensor-core rate probe (peak.cu): ops of one launch (0: unsupported kind / n) and its launcher
+double mma_rate_ops(int kind, int n, int iters, int ctas);
+cudaError_t launch_mma_rate(int kind, int n, int iters, int ctas, cudaStream_t st);
 cudaError_t launch_quant_nvfp4(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st);
 // kernels (not counting memsets) that launch_quant_nvfp4 enqueues for a's sizes and flags
 int quant_nvfp4_kernel_count(const QuantArgs& a, int is_fp16, bool allow_one_read);

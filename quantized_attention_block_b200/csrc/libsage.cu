@@ -5,5 +5,6 @@
 #include "attn_i8f8.cu"
 #include "quant_nvfp4.cu"
 #include "attn_nvfp4.cu"
+#include "peak.cu"
 #include "api.cu"
 #include "noalloc.cu"

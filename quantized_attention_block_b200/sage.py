@@ -29,7 +29,7 @@ EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized",
             "sage_nvfp4_workspace_bytes", "sage_quant_nvfp4", "sage_attn_fwd_nvfp4_quantized",
             "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4", "sage_debug_exp2_poly",
             "sage_debug_kv_quant_two_pass", "sage_quant_kernel_count", "sage_quant_nvfp4_kernel_count",
-            "sage_attn_fwd_quantized_lse", "sage_attn_fwd_lse")
+            "sage_attn_fwd_quantized_lse", "sage_attn_fwd_lse", "sage_debug_mma_rate")
 
 
 class SageError(RuntimeError):
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.sage_debug_qk_nvfp4.argtypes = [F, P, i32, i32, i32, i32, vp, vp]
         L.sage_debug_exp2_poly.argtypes, L.sage_debug_exp2_poly.restype = [vp, vp, i32, vp], ctypes.c_int
         L.sage_debug_kv_quant_two_pass.argtypes, L.sage_debug_kv_quant_two_pass.restype = [i32], ctypes.c_int
+        L.sage_debug_mma_rate.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp]
+        L.sage_debug_mma_rate.restype = ctypes.c_int
         L.sage_quant_kernel_count.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         L.sage_quant_kernel_count.restype = ctypes.c_int
         L.sage_quant_nvfp4_kernel_count.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
@@ -319,6 +321,18 @@ def sage_debug_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
     y = torch.empty_like(x)
     _check(lib().sage_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "sage_debug_exp2_poly")
     return y
+
+
+MMA_KINDS = {"i8": 0, "f8": 1, "f4": 2}
+
+
+def sage_debug_mma_rate(kind: str, n: int, iters: int, ctas: int = 0, stream=None) -> float:
+    """Enqueue the tensor-core rate probe (one CTA per SM by default) on `stream`
+    and return the operation count of that launch; time it with CUDA events."""
+    ops = ctypes.c_double(0.0)
+    _check(lib().sage_debug_mma_rate(MMA_KINDS[kind], int(n), int(iters), int(ctas), ctypes.byref(ops),
+                                     _stream(stream)), "sage_debug_mma_rate")
+    return float(ops.value)
 
 
 def sage_quant_kernel_count(p: SageParams) -> int:
