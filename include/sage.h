@@ -152,7 +152,11 @@ SAGE_API sage_status sage_quant_qkv(const void *q, const void *k, const void *v,
 SAGE_API sage_status sage_attn_fwd_quantized(const sage_quant_view *view, void *o, const sage_params *p,
                                     void *stream);
 
-/* sage_quant_qkv followed by sage_attn_fwd_quantized (the whole forward). */
+/* sage_quant_qkv followed by sage_attn_fwd_quantized (the whole forward).
+ * Both attention kernels check the device error word first: while an error
+ * recorded by an earlier launch (a quantiser wait that ran out and left codes
+ * unwritten) has not been read by sage_last_device_error, they return without
+ * touching `o`, so O is never computed from stale codes. */
 SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, void *o, const sage_params *p,
                           void *workspace, size_t workspace_bytes, void *stream);
 
@@ -361,10 +365,21 @@ SAGE_API sage_status sage_quant_nvfp4_kernel_count(const sage_params *p, int32_t
 /*
  * Test hook: on = 1 makes sage_quant_qkv and sage_quant_nvfp4 (and the calls
  * built on them) take the two-pass K/V path (statistics kernel, then the code
- * kernels) in this process; on = 0 restores the default choice.  Not thread-safe with
- * concurrent sage_quant_qkv calls.  SAGE_ERR_INVALID_ARG for other values.
+ * kernels) in this process; on = 2 makes them take the one-read path even when
+ * a (head, K|V) group's tiles may not all be resident at once, so that its
+ * bounded waits can run out (a test of the timeout path: the waits give up,
+ * SAGE_ERR_TIMEOUT is recorded, the tiles that gave up write no codes); on = 0
+ * restores the default choice.  Not thread-safe with concurrent
+ * sage_quant_qkv calls.  SAGE_ERR_INVALID_ARG for other values.
  */
 SAGE_API sage_status sage_debug_kv_quant_two_pass(int32_t on);
+
+/*
+ * Test hook: the limit of every bounded in-kernel wait, in microseconds, for
+ * the launches enqueued after this call on `stream` (0 restores the default of
+ * 4 s).  Synchronises `stream`.  1 <= timeout_us <= 10 s, or 0.
+ */
+SAGE_API sage_status sage_debug_wait_limit(uint32_t timeout_us, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 SAGE_API const char *sage_status_string(sage_status s);

@@ -30,7 +30,9 @@ struct Layout {
   size_t q8, k8, v8t, s_q, s_k, s_v, km, qkm, ksum, vamax, kv_sync, kv_sync_end, qbar, dS, total;
 };
 
-// 1: sage_quant_qkv always takes the two-pass K/V path (sage_debug_kv_quant_two_pass)
+// K/V path of sage_quant_qkv / sage_quant_nvfp4 (sage_debug_kv_quant_two_pass):
+// 0: the default choice; 1: always two passes; 2: one read even when a group's
+// tiles may not all be resident at once (a test of the bounded group waits)
 int g_kv_two_pass = 0;
 
 sage_status check_params(const sage_params* p, Dims* d) {
@@ -363,7 +365,8 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, const sa
   a.qkm = view->qkm;
   a.ksum = reinterpret_cast<double*>(base + L.ksum);
   a.vamax = reinterpret_cast<unsigned*>(base + L.vamax);
-  a.kv_sync = g_kv_two_pass ? nullptr : reinterpret_cast<int*>(base + L.kv_sync);
+  a.kv_sync = g_kv_two_pass == 1 ? nullptr : reinterpret_cast<int*>(base + L.kv_sync);
+  a.force_one_read = g_kv_two_pass == 2;
   a.kv_zero_bytes = L.kv_sync_end - L.ksum;
   QuantMaps m;
   if (!map_2d_u8(&m.vt, view->v8t, (uint64_t)d.Np, (uint64_t)(d.B * d.Hkv * d.D), kTile, (uint32_t)d.D,
@@ -482,7 +485,8 @@ sage_status sage_quant_nvfp4(const void* q, const void* k, const void* v, const 
   a.sfq = view->sfq;
   a.sfk = view->sfk;
   a.sfv = view->sfv;
-  a.kv_sync = g_kv_two_pass ? nullptr : reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + L.kv_sync);
+  a.kv_sync = g_kv_two_pass == 1 ? nullptr : reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + L.kv_sync);
+  a.force_one_read = g_kv_two_pass == 2;
   a.kv_zero_bytes = L.kv_sync_end - L.ksum;
   QuantMaps m;
   if (!map_input(&m.q, q, (uint64_t)d.D, (uint64_t)d.N, (uint64_t)d.Hq, (uint64_t)d.B, p->layout) ||
@@ -589,7 +593,8 @@ sage_status sage_quant_kernel_count(const sage_params* p, int32_t* n) {
   a.bk = p->bk;
   a.smooth_k = p->smooth_k;
   a.smooth_q = p->smooth_q;
-  *n = quant_kernel_count(a, p->dtype == SAGE_FP16, g_kv_two_pass == 0);
+  a.force_one_read = g_kv_two_pass == 2;
+  *n = quant_kernel_count(a, p->dtype == SAGE_FP16, g_kv_two_pass != 1);
   return SAGE_OK;
 }
 
@@ -612,14 +617,27 @@ sage_status sage_quant_nvfp4_kernel_count(const sage_params* p, int32_t* n) {
   a.bk = p->bk;
   a.smooth_k = p->smooth_k;
   a.smooth_q = p->smooth_q;
-  *n = quant_nvfp4_kernel_count(a, p->dtype == SAGE_FP16, g_kv_two_pass == 0);
+  a.force_one_read = g_kv_two_pass == 2;
+  *n = quant_nvfp4_kernel_count(a, p->dtype == SAGE_FP16, g_kv_two_pass != 1);
   return SAGE_OK;
 }
 
 sage_status sage_debug_kv_quant_two_pass(int32_t on) {
-  if (on != 0 && on != 1) return SAGE_ERR_INVALID_ARG;
+  if (on < 0 || on > 2) return SAGE_ERR_INVALID_ARG;
   g_kv_two_pass = on;
   return SAGE_OK;
+}
+
+sage_status sage_debug_wait_limit(uint32_t timeout_us, void* stream) {
+  if (timeout_us > 10u * 1000u * 1000u) return SAGE_ERR_INVALID_ARG;
+  sage_status s = check_arch();
+  if (s != SAGE_OK) return s;
+  const unsigned long long limit = timeout_us ? 1000ull * timeout_us : 4000000000ull;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyToSymbolAsync(sage::g_wait_limit_ns, &limit, sizeof(limit), 0, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return SAGE_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
 sage_status sage_debug_exp2_poly(const float* x, float* y, int32_t n, void* stream) {

@@ -160,6 +160,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   bar.mma_done = bar.o_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oTmem);
 
+  // An unread device error (a quantiser wait that ran out leaves some codes
+  // unwritten) stops the launch before it reads the quantised tensors: O is
+  // left as it was rather than computed from stale codes.
+  __shared__ int s_skip;
+  if (threadIdx.x == 0) s_skip = device_error_pending() ? 1 : 0;
+  __syncthreads();
+  if (s_skip) return;
+
   // ---- work: (b, h, pair of Q tiles), heavy causal pairs first
   const int bhq = a.B * a.Hq;
   const int n_pairs = (a.n_qtiles + 1) / 2;

@@ -47,6 +47,8 @@ struct QuantArgs {
                          // NVFP4 path (K only)
   size_t kv_zero_bytes;  // bytes from ksum through the end of kv_sync (consecutive in
                          // the workspace), zeroed before the one-read kernel
+  int force_one_read;    // test hook: take the one-read path even when a group's tiles may
+                         // not all be resident at once (its bounded waits then run out)
   // NVFP4 path (E2M1 codes two per byte, low nibble first; 1 KB scale blocks
   // per 128-row tile in the tcgen05 scale-factor order)
   uint8_t* q4;   // [B,Hq,Np,D/2]

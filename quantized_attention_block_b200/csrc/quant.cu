@@ -879,7 +879,7 @@ void (*kv_fused_kernel(const QuantArgs& a, int tiles, int smem))(CUtensorMap, CU
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kf, kThreads, smem) != cudaSuccess)
     return nullptr;
-  return (int64_t)tiles * 2 <= (int64_t)sms * per_sm ? kf : nullptr;
+  return (a.force_one_read || (int64_t)tiles * 2 <= (int64_t)sms * per_sm) ? kf : nullptr;
 }
 
 template <typename T, int D, bool QKM>

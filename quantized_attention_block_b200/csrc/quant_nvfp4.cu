@@ -287,7 +287,7 @@ KNvfp4Fn k_fused_nvfp4_for(const QuantArgs& a, int tiles, int smem) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kf, kThreads, smem) != cudaSuccess)
     return nullptr;
-  return (int64_t)tiles * 2 <= (int64_t)sms * per_sm ? kf : nullptr;
+  return (a.force_one_read || (int64_t)tiles * 2 <= (int64_t)sms * per_sm) ? kf : nullptr;
 }
 
 template <typename T>

@@ -23,6 +23,12 @@ __device__ __forceinline__ void record_error(unsigned int code) {
   atomicCAS(&g_device_error, 0u, code);
 }
 
+// An error recorded by an earlier kernel (e.g. a quantiser's wait that ran out)
+// and not yet read by the host.
+__device__ __forceinline__ bool device_error_pending() {
+  return *reinterpret_cast<volatile unsigned int*>(&g_device_error) != 0u;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -59,6 +65,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Test of the phase with parity `parity` that may suspend the thread for up to
+// about `hint_ns` while the phase is incomplete (a waiting warp issues nothing).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }

@@ -29,7 +29,8 @@ EXPORTED = ("sage_workspace_bytes", "sage_quant_qkv", "sage_attn_fwd_quantized",
             "sage_nvfp4_workspace_bytes", "sage_quant_nvfp4", "sage_attn_fwd_nvfp4_quantized",
             "sage_attn_fwd_nvfp4", "sage_debug_qk_nvfp4", "sage_debug_exp2_poly",
             "sage_debug_kv_quant_two_pass", "sage_quant_kernel_count", "sage_quant_nvfp4_kernel_count",
-            "sage_attn_fwd_quantized_lse", "sage_attn_fwd_lse", "sage_debug_mma_rate")
+            "sage_attn_fwd_quantized_lse", "sage_attn_fwd_lse", "sage_debug_mma_rate",
+            "sage_debug_wait_limit")
 
 
 class SageError(RuntimeError):
@@ -100,6 +101,7 @@ def lib() -> ctypes.CDLL:
         L.sage_debug_kv_quant_two_pass.argtypes, L.sage_debug_kv_quant_two_pass.restype = [i32], ctypes.c_int
         L.sage_debug_mma_rate.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp]
         L.sage_debug_mma_rate.restype = ctypes.c_int
+        L.sage_debug_wait_limit.argtypes, L.sage_debug_wait_limit.restype = [ctypes.c_uint32, vp], ctypes.c_int
         L.sage_quant_kernel_count.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         L.sage_quant_kernel_count.restype = ctypes.c_int
         L.sage_quant_nvfp4_kernel_count.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
@@ -349,9 +351,16 @@ def sage_quant_nvfp4_kernel_count(p: SageParams) -> int:
     return int(n.value)
 
 
-def sage_debug_kv_quant_two_pass(on: bool) -> None:
-    """Force (True) or release (False) the two-pass K/V quantisation path in this process."""
-    _check(lib().sage_debug_kv_quant_two_pass(1 if on else 0), "sage_debug_kv_quant_two_pass")
+def sage_debug_kv_quant_two_pass(on) -> None:
+    """Force (True / 1) or release (False / 0) the two-pass K/V quantisation path in
+    this process; 2 forces the one-read path even when a group's tiles may not
+    all be resident (a test of its bounded waits)."""
+    _check(lib().sage_debug_kv_quant_two_pass(int(on)), "sage_debug_kv_quant_two_pass")
+
+
+def sage_debug_wait_limit(timeout_us: int, stream=None) -> None:
+    """Limit of the in-kernel bounded waits for later launches (0: the default 4 s)."""
+    _check(lib().sage_debug_wait_limit(int(timeout_us), _stream(stream)), "sage_debug_wait_limit")
 
 
 def nvfp4_view_tensors(view: SageNvfp4View, p: SageParams, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:
