@@ -666,6 +666,573 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Split-row variant, taken when delta_S is added (smooth Q).  Folding delta_S
+// into the scores costs every score another FMA and a shared-memory read in
+// the softmax, whose instruction stream bounds the kernel; here each 128-key
+// tile of a Q row is split between two warps, so twice the warps share that
+// work.  640 threads in five warpgroups:
+//   WG0      warp 0: TMA producer; warp 1: MMA issuer and TMEM owner
+//   WG1, 2   Q tile 0, key columns [0, 64) and [64, 128) of every K tile, and
+//            O columns [0, D/2) and [D/2, D) (rescale / level-2 sum, epilogue)
+//   WG3, 4   the same for Q tile 1
+// The two warps on the same 32 TMEM lanes (one row each per thread) exchange
+// their half-row maxima through shared memory, so both quantise P with the
+// row's maximum; their row sums are added at the end.  The schedule, the
+// TMEM layout and the shared-memory operands are those of the kernel above;
+// without delta_S that kernel is faster (its exchange-free rows beat the
+// halved work).
+constexpr int kThreadsSplit = 640;
+
+// per-warpgroup register budgets of the split-row kernel after setmaxnreg (640 threads launch with
+// 96 registers each; the five warpgroups must not ask for more in total)
+constexpr uint32_t kRegsSplitProducer = 32, kRegsSplitSoftmax = 112;
+static_assert(kRegsSplitProducer + 4 * kRegsSplitSoftmax <= 5 * 96, "register split exceeds the launch");
+
+template <int D>
+struct SmemSplit {
+  static constexpr uint32_t kQ = 128 * D, kK = 128 * D, kV = D * 128, kP = 128 * 128;  // kP: one P buffer
+  static constexpr uint32_t oQ = 0;                      // 2 tiles
+  static constexpr uint32_t oK = oQ + 2 * kQ;            // kStages
+  static constexpr uint32_t oV = oK + kStages * kK;      // kStages
+  static constexpr uint32_t oP = oV + kStages * kV;      // [tile][2 buffers]
+  static constexpr uint32_t kDS = 2 * 4 * 128 * 4;      // delta_S rows of one key tile: [tile][Q block (<= 4)][128]
+  static constexpr uint32_t oDS = oP + 4 * kP;           // kStages
+  static constexpr uint32_t oMx = oDS + kStages * kDS;   // float[buffer j & 1][tile][half][128] half-row maxima
+  static constexpr uint32_t oL = oMx + 2 * 2 * 2 * 128 * 4;  // float[tile][half][128] l, then [tile][128] m
+  static constexpr uint32_t oBar = oL + (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr uint32_t kNumBars = 1 + 3 * kStages + 2 + 4 + 4 + 2 + 2 + 2 + 1 + 16 + 8;
+  static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
+  static constexpr uint32_t kBytes = oTmem + 16 + 1024;  // + alignment slack
+  static_assert(kBytes <= 227 * 1024, "attention tile buffers exceed the shared memory of one CTA");
+};
+
+struct BarsSplit {
+  uint64_t* q_full;
+  uint64_t* k_full;    // [kStages]  K_j (+ delta_S rows) landed
+  uint64_t* v_full;    // [kStages]
+  uint64_t* kv_empty;  // [kStages]
+  uint64_t* s_full;    // [2]  QK^T of tile i done            (tcgen05.commit)
+  uint64_t* p_full;    // [tile][buffer j & 1]  P_i(j) written (one arrival per softmax warp of the
+                       //      tile, 8); one barrier per buffer keeps every waiter at most one phase behind
+  uint64_t* p_empty;   // [tile][buffer]  the P V that read that P buffer retired (tcgen05.commit)
+  uint64_t* ot_full;   // [2]  P V of tile i retired              (tcgen05.commit)
+  uint64_t* r_free;    // [2]  S_i columns hold the magic fill again and may take the next QK^T
+                       //      (TMEM accumulator: S read; two-level: O_t read); one arrival per warp
+  uint64_t* o_ready;   // [2]  (TMEM accumulator mode) O_i rescaled by alpha_i(j) for P V(i, j); one
+                       //      arrival per softmax warp, every j
+  uint64_t* mma_done;  // all tensor-core work of the CTA retired (one commit at the end)
+  uint64_t* mx;        // [tile][lane quarter][buffer j & 1]  both halves of these rows posted their
+                       //      maximum of tile j (one arrival per warp, 2)
+  uint64_t* lx;        // [tile][lane quarter]  both halves posted their row sums (2)
+};
+
+// LSE: also write each row's log-sum-exp (a separate instance, so that kernels
+// without it carry none of its code)
+template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO, bool LSE>
+__global__ void __launch_bounds__(kThreadsSplit, 1)
+    attn_i8f8_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  using L = SmemSplit<D>;
+  constexpr uint32_t kSwzQK = (D == 128) ? kSwizzle128B : kSwizzle64B;
+  constexpr uint32_t kSboQK = 8 * D;  // 8 rows x D bytes per swizzle atom
+  constexpr uint32_t kIdescQK = make_idesc(/*S32*/ 2, /*s8*/ 1, /*s8*/ 1, 128, 128);
+  constexpr uint32_t kIdescPV = make_idesc(/*F32*/ 1, /*E4M3*/ 0, /*E4M3*/ 0, 128, D);
+  constexpr uint32_t kTmemCols = 512;
+  constexpr int DH = D / 2;  // O columns per softmax half
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem + L::oQ;
+  uint8_t* sK = smem + L::oK;
+  uint8_t* sV = smem + L::oV;
+  uint8_t* sP = smem + L::oP;
+  const float* sDS = reinterpret_cast<const float*>(smem + L::oDS);
+  float* s_mx = reinterpret_cast<float*>(smem + L::oMx);
+  float* s_l = reinterpret_cast<float*>(smem + L::oL);
+  uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L::oBar);
+  BarsSplit bar;
+  bar.q_full = bar0;
+  bar.k_full = bar0 + 1;
+  bar.v_full = bar.k_full + kStages;
+  bar.kv_empty = bar.v_full + kStages;
+  bar.s_full = bar.kv_empty + kStages;
+  bar.p_full = bar.s_full + 2;
+  bar.p_empty = bar.p_full + 4;
+  bar.ot_full = bar.p_empty + 4;
+  bar.r_free = bar.ot_full + 2;
+  bar.o_ready = bar.r_free + 2;
+  bar.mma_done = bar.o_ready + 2;
+  bar.mx = bar.mma_done + 1;
+  bar.lx = bar.mx + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oTmem);
+
+  // An unread device error (a quantiser wait that ran out leaves some codes
+  // unwritten) stops the launch before it reads the quantised tensors: O is
+  // left as it was rather than computed from stale codes.
+  __shared__ int s_skip;
+  if (threadIdx.x == 0) s_skip = device_error_pending() ? 1 : 0;
+  __syncthreads();
+  if (s_skip) return;
+
+  // ---- work: (b, h, pair of Q tiles), heavy causal pairs first
+  const int bhq = a.B * a.Hq;
+  const int n_pairs = (a.n_qtiles + 1) / 2;
+  const int pr = n_pairs - 1 - (int)(blockIdx.x / bhq);
+  const int bh = blockIdx.x % bhq;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const int g = h / (a.Hq / a.Hkv);
+  const int n_kt = (int)(a.Np / kTile);
+  int nTi[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int qt = 2 * pr + i;
+    nTi[i] = qt >= a.n_qtiles ? 0 : (CAUSAL ? qt + 1 : n_kt);
+  }
+  const int nT = nTi[0] > nTi[1] ? nTi[0] : nTi[1];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int wg = warp / 4;
+  if (threadIdx.x == 0) {
+    mbar_init(bar.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.s_full[i], 1);
+      mbar_init(&bar.ot_full[i], 1);
+      mbar_init(&bar.r_free[i], 8);
+      mbar_init(&bar.o_ready[i], 8);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bar.p_full[i], 8);
+      mbar_init(&bar.p_empty[i], 1);
+    }
+    mbar_init(bar.mma_done, 1);
+    for (int i = 0; i < 16; ++i) mbar_init(&bar.mx[i], 2);
+    for (int i = 0; i < 8; ++i) mbar_init(&bar.lx[i], 2);
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // S accumulators start at the int32 bit pattern of 1.5 * 2^23: QK^T accumulates
+  // onto it, so TMEM returns 0x4B400000 + acc, which read as fp32 is exactly
+  // 12582912 + acc (|acc| <= 127 * 127 * 128 < 2^22): no int -> float step.
+  // Each softmax warp fills (and later refills) its half of its tile's columns.
+  if (wg >= 1) {
+    const int ti = (wg - 1) >> 1, hf = (wg - 1) & 1;
+    const uint32_t tS0 = tmem + 128 * ti + 64 * hf + ((uint32_t)((warp & 3) * 32) << 16);
+#pragma unroll
+    for (int c = 0; c < 64; c += 8) tmem_fill8(tS0 + c, kMagicBits);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (wg == 0) {
+    regs_dec<kRegsSplitProducer>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+      const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
+      const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np);
+      const int vrow = (b * a.Hkv + g) * D;
+      const int ds_rows = kTile / a.bq;  // Q blocks per tile (1, 2 or 4)
+      const uint32_t ds_bytes = (uint32_t)((nTi[0] > 0) + (nTi[1] > 0)) * ds_rows * 512;
+      mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
+      for (int i = 0; i < 2; ++i)
+        if (nTi[i] > 0) tma_load_2d(sQ + i * L::kQ, &tmQ, bar.q_full, 0, (int)(qhead + (int64_t)(2 * pr + i) * kTile));
+      bool ok = true;
+      int j = 0;
+      for (; j < nT && ok; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages) ok = mbar_wait(&bar.kv_empty[s], ((j / kStages) + 1) & 1);
+        if (!ok) break;
+        mbar_expect_tx(&bar.k_full[s], L::kK + (HAS_DS ? ds_bytes : 0u));
+        tma_load_2d(sK + s * L::kK, &tmK, &bar.k_full[s], 0, krow0 + j * kTile);
+        if (HAS_DS) {
+          // delta_S[b, h, Q block, keys of tile j] for the Q blocks of both tiles
+          for (int i = 0; i < 2; ++i)
+            for (int hb = 0; hb < ds_rows; ++hb)
+              if (nTi[i] > 0) {
+                const int blk = min((2 * pr + i) * ds_rows + hb, a.Tm - 1);
+                bulk_load_1d(smem + L::oDS + s * L::kDS + (i * 4 + hb) * 512,
+                             a.dS + ((int64_t)(b * a.Hq + h) * a.Tm + blk) * a.Np + (int64_t)j * kTile, 512,
+                             &bar.k_full[s]);
+              }
+        }
+        mbar_expect_tx(&bar.v_full[s], L::kV);
+        tma_load_2d(sV + s * L::kV, &tmV, &bar.v_full[s], j * kTile, vrow);
+      }
+      // never leave a copy in flight
+      for (int jj = (j - kStages > 0 ? j - kStages : 0); jj < j; ++jj) {
+        mbar_wait(&bar.k_full[jj % kStages], (jj / kStages) & 1);
+        mbar_wait(&bar.v_full[jj % kStages], (jj / kStages) & 1);
+      }
+      mbar_wait(bar.q_full, 0);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t aP0 = smem_u32(sP);
+        bool ok = mbar_wait(bar.q_full, 0);
+        auto issue_qk = [&](int i, int j) {
+          const int s = j % kStages;
+          const uint32_t aQ = smem_u32(sQ + i * L::kQ), aK = smem_u32(sK + s * L::kK);
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_i8(tmem + 128 * i, make_sdesc(aQ + kk * 32, kSboQK, kSwzQK), make_sdesc(aK + kk * 32, kSboQK, kSwzQK),
+                   kIdescQK, 1u);  // accumulate onto the magic fill
+          mma_commit(&bar.s_full[i]);
+        };
+        auto issue_pv = [&](int i, int j) {
+          const int s = j % kStages;
+          const uint32_t aP = aP0 + (i * 2 + (j & 1)) * L::kP, aV = smem_u32(sV + s * L::kV);
+          // two-level: a fresh O_t tile in S_i's columns; else accumulate into O_i
+          const uint32_t dst = TWO_LEVEL ? tmem + 128 * i : tmem + 256 + D * i;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 32; ++kk)
+            mma_f8f6f4(dst, make_sdesc(aP + kk * 32, 1024, kSwizzle128B), make_sdesc(aV + kk * 32, 1024, kSwizzle128B),
+                       kIdescPV, (kk > 0 || (!TWO_LEVEL && j > 0)) ? 1u : 0u);
+          mma_commit(&bar.ot_full[i]);
+          mma_commit(&bar.p_empty[i * 2 + (j & 1)]);
+        };
+        // Two independent per-tile chains, each op issued as soon as its inputs
+        // are ready (non-blocking polls), so one tile never holds the other back.
+        //   QK(i,j): K_j landed; j > 0: S_i columns refilled (r_free) and, two-level,
+        //            PV(i,j-1) issued (its O_t shares those columns)
+        //   PV(i,j): QK(i,j) issued; V_j landed; P_i(j) written; TMEM-accumulator
+        //            mode: O_i rescaled by alpha_i(j) (o_ready phase j)
+        // Stage j of the K/V ring is released once every active tile issued PV(i,j).
+        int next_qk[2] = {0, 0}, next_pv[2] = {0, 0};
+        int released = 0;
+        uint64_t t_idle = 0;
+        while (ok) {
+          bool progress = false;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int jq = next_qk[i], jp = next_pv[i];
+            if (jq < nTi[i] && (!TWO_LEVEL || jp >= jq) &&
+                mbar_test_wait(smem_u32(&bar.k_full[jq % kStages]), (jq / kStages) & 1) &&
+                (jq == 0 || mbar_test_wait(smem_u32(&bar.r_free[i]), (jq - 1) & 1))) {
+              tc_fence_after();
+              issue_qk(i, jq);
+              next_qk[i] = jq + 1;
+              progress = true;
+            }
+            if (jp < nTi[i] && next_qk[i] > jp &&
+                mbar_test_wait(smem_u32(&bar.p_full[i * 2 + (jp & 1)]), (jp >> 1) & 1) &&
+                mbar_test_wait(smem_u32(&bar.v_full[jp % kStages]), (jp / kStages) & 1) &&
+                (TWO_LEVEL || mbar_test_wait(smem_u32(&bar.o_ready[i]), jp & 1))) {
+              tc_fence_after();
+              issue_pv(i, jp);
+              next_pv[i] = jp + 1;
+              progress = true;
+            }
+          }
+          while (released < nT && (next_pv[0] > released || released >= nTi[0]) &&
+                 (next_pv[1] > released || released >= nTi[1])) {
+            mma_commit(&bar.kv_empty[released % kStages]);
+            ++released;
+          }
+          if (next_pv[0] >= nTi[0] && next_pv[1] >= nTi[1] && released >= nT) break;
+          // spin (a sleep here delays the reaction to a ready operand), bounded by the idle time
+          if (progress) {
+            t_idle = 0;
+          } else if (t_idle == 0) {
+            t_idle = globaltimer_ns();
+          } else if (globaltimer_ns() - t_idle > g_wait_limit_ns) {
+            record_error(kDevErrTimeout);
+            ok = false;
+          }
+        }
+        // every tensor-core op retired before TMEM is released
+        mma_commit(bar.mma_done);
+        mbar_wait(bar.mma_done, 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ softmax, accumulation, epilogue
+    // Warpgroups 1, 2 take Q tile 0 and 3, 4 tile 1; within a tile warpgroup
+    // hf = 0 owns key columns [0, 64) of every 128-key tile and O columns
+    // [0, D/2), hf = 1 the other halves.  A thread owns one Q row (one TMEM
+    // lane) in both; the two halves of a row exchange their maxima through
+    // shared memory (an mbarrier of the two warps on the same 32 lanes), so
+    // both quantise P with the same row max, and add their partial row sums
+    // at the end.
+    regs_inc<kRegsSplitSoftmax>();
+    const int ti = (wg - 1) >> 1;  // Q tile
+    const int hf = (wg - 1) & 1;   // column half
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int qtile = 2 * pr + ti;
+    const int64_t qrow = (int64_t)qtile * kTile + row;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + 128 * ti + 64 * hf + lane_off;  // this half's 64 S columns
+    const uint32_t tO = tmem + 256 + D * ti + DH * hf + lane_off;  // this half's D/2 O columns
+    uint64_t* mxbar = bar.mx + (ti * 4 + quarter) * 2;  // the two warps on these lanes, per buffer
+    const int qblk = min((int)(qrow / a.bq), a.Tm - 1);
+    const float row_scale = a.s_q[(int64_t)(b * a.Hq + h) * a.Tm + qblk] * a.scale_log2;
+    const float* sk = a.s_k + (int64_t)(b * a.Hkv + g) * a.Tn;
+    // this row's Q block within the tile (warp-uniform: bq >= 32); a shift, not a
+    // division by the runtime bq (which the compiler would redo in the tile loop)
+    const int ds_blk = row >> (a.bq == 32 ? 5 : (a.bq == 64 ? 6 : 7));
+    // key-block scale of this half's 64 keys (bk = 64: one block; bk = 128: the tile's)
+    float sk_h = __ldg(sk + min((64 * hf) / a.bk, a.Tn - 1));
+    const float sl2 = a.scale_log2;
+    const float2 neg_magic = make_float2(-kMagic, -kMagic);
+    float m = -INFINITY, l = 0.0f;
+    bool ok = true;
+    uint32_t x[32];
+
+    for (int j = 0; j < nTi[ti] && ok; ++j) {
+      if (!(ok = mbar_wait_warp(&bar.s_full[ti], j & 1))) break;
+      tc_fence_after();
+      uint32_t s[64];  // fp32 bits of y = 12582912 + acc (acc = the INT8 dot product)
+      tmem_ld32p(tS + 0, s + 0);
+      tmem_ld32p(tS + 32, s + 32);
+      const int col0 = j * kTile + 64 * hf;
+      // a = s_q s_k sm_scale log2 e of this half's keys, kept > 0 so that a masked
+      // -inf stays -inf (a zero scale only multiplies zero dot products)
+      const float a_h = fmaxf(row_scale * sk_h, FLT_MIN);
+      // next tile's key-block scale (its load latency hides behind this tile)
+      sk_h = __ldg(sk + min((j * kTile + kTile + 64 * hf) / a.bk, a.Tn - 1));
+      const float* dsr = sDS + (j % kStages) * (L::kDS / 4) + (ti * 4 + ds_blk) * 128 + 64 * hf;
+      if (HAS_DS && !(ok = mbar_wait_warp(&bar.k_full[j % kStages], (j / kStages) & 1))) break;
+      tmem_ld_wait();
+      if (!TWO_LEVEL) {
+        // S_i is in registers: restore the magic fill, then the next QK^T may run
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) tmem_fill8(tS + c, kMagicBits);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.r_free[ti]);
+      }
+      const bool need_mask = (j * kTile + kTile > a.N) || (CAUSAL && j == qtile);
+      // with delta_S: x = (y - 12582912) + delta_S sm_scale log2 e / a in place, so
+      // that the score is t = x a (a >= 1e-30 here keeps the quotient finite)
+      const float ad = fmaxf(a_h, 1e-30f);
+      if (HAS_DS) {
+        const float kc = sl2 / ad;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const float4 ds = *reinterpret_cast<const float4*>(dsr + c);
+          const float2 x0 = ffma2(make_float2(ds.x, ds.y), make_float2(kc, kc),
+                                  fadd2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), neg_magic));
+          const float2 x1 = ffma2(make_float2(ds.z, ds.w), make_float2(kc, kc),
+                                  fadd2(make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])), neg_magic));
+          s[c] = __float_as_uint(x0.x);
+          s[c + 1] = __float_as_uint(x0.y);
+          s[c + 2] = __float_as_uint(x1.x);
+          s[c + 3] = __float_as_uint(x1.y);
+        }
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int col = col0 + c;
+          if (col >= a.N || (CAUSAL && col > qrow)) s[c] = __float_as_uint(-INFINITY);
+        }
+      }
+      // max of this half (on the raw values: x, or y, is monotonic in the score)
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
+      const float mraw = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+      const float mx_h = HAS_DS ? mraw * ad : (mraw - kMagic) * a_h;
+      // the row max over both halves (the partner warp's value of this tile)
+      float* mxb = s_mx + (j & 1) * 512 + ti * 256;
+      mxb[hf * 128 + row] = mx_h;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mxbar[j & 1]);
+      if (!(ok = mbar_wait_warp(&mxbar[j & 1], (j >> 1) & 1))) break;
+      const float m_new = fmaxf(m, fmaxf(mx_h, mxb[(1 - hf) * 128 + row]));
+      const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
+      const float mm = (m_new == -INFINITY) ? 0.0f : m_new - kLog2_448;
+      // P buffer (j & 1) is free once P V(j - 2) retired
+      if (j >= 2 && !(ok = mbar_wait_warp(&bar.p_empty[ti * 2 + (j & 1)], ((j >> 1) - 1) & 1))) break;
+      uint8_t* myP = sP + (ti * 2 + (j & 1)) * L::kP + row * 128;
+      // P = exp2(t - m + log2 448) -> E4M3 -> shared memory (128B-swizzled K-major);
+      // this half writes 16-byte chunks 4 hf .. 4 hf + 3 of its row
+      float2 rs[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rs[k] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const int c = grp * 16 + e;
+          float2 u0, u1;
+          const float2 y0 = make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          const float2 y1 = make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+          if (HAS_DS) {
+            u0 = ffma2(y0, make_float2(ad, ad), make_float2(-mm, -mm));
+            u1 = ffma2(y1, make_float2(ad, ad), make_float2(-mm, -mm));
+          } else {
+            u0 = ffma2(fadd2(y0, neg_magic), make_float2(a_h, a_h), make_float2(-mm, -mm));
+            u1 = ffma2(fadd2(y1, neg_magic), make_float2(a_h, a_h), make_float2(-mm, -mm));
+          }
+          const float2 p0 = make_float2(ex2_approx(u0.x), ex2_approx(u0.y));
+          const float2 p1 = make_float2(ex2_approx(u1.x), ex2_approx(u1.y));
+          rs[e / 4] = fadd2(rs[e / 4], fadd2(p0, p1));
+          w[e / 4] = cvt_e4m3x4(p0.x, p0.y, p1.x, p1.y);
+        }
+        *reinterpret_cast<uint4*>(myP + (((4 * hf + grp) ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      const float2 rs2 = fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3]));
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.p_full[ti * 2 + (j & 1)]);
+      l = fmaf(l, alpha, rs2.x + rs2.y);
+      m = m_new;
+      if constexpr (TWO_LEVEL) {
+        // level 2 on this half of O_i: O = alpha O + O_t, where P V(j) put a fresh
+        // O_t into S_i's columns [0, D).  O_t is read first, then S_i's columns of
+        // this half get the magic fill back (this half's O_t columns and, for
+        // D = 64, its share of the columns O_t does not cover) and the next QK^T
+        // may run while the sum is formed.
+        if (!(ok = mbar_wait_warp(&bar.ot_full[ti], j & 1))) break;
+        tc_fence_after();
+        const uint32_t tOt = tmem + 128 * ti + DH * hf + lane_off;
+        uint32_t* ot = s;  // S is consumed: its registers take O_t
+#pragma unroll
+        for (int c = 0; c < DH; c += 32) tmem_ld32p(tOt + c, ot + c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < DH; c += 8) tmem_fill8(tOt + c, kMagicBits);
+        if (D < 128) {
+#pragma unroll
+          for (int c = 0; c < (128 - D) / 2; c += 8) tmem_fill8(tmem + 128 * ti + D + (128 - D) / 2 * hf + lane_off + c, kMagicBits);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.r_free[ti]);
+#pragma unroll
+        for (int c = 0; c < DH; c += 32) {
+          if (j == 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = ot[c + e];
+          } else {
+            tmem_ld32(tO + c, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 o = ffma2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])),
+                                     make_float2(alpha, alpha),
+                                     make_float2(__uint_as_float(ot[c + e]), __uint_as_float(ot[c + e + 1])));
+              x[e] = __float_as_uint(o.x);
+              x[e + 1] = __float_as_uint(o.y);
+            }
+          }
+          tmem_st32(tO + c, x);
+        }
+        tmem_st_wait();
+      } else {
+        // O_i accumulates in TMEM; before P V(i, j) adds tile j, this half's columns
+        // of rows whose max grew are rescaled by alpha = e^(m_old - m_new) (a warp
+        // whose 32 rows all have alpha == 1 leaves them untouched: exact).  P V(i, j - 1)
+        // must have retired first, and is waited for even when nothing is rescaled:
+        // o_ready(j + 1) then cannot complete before P V(i, j) was issued, so the
+        // issuer's parity test of o_ready never sees it two phases ahead.  o_ready is
+        // signalled for every j (P V(i, 0) waits for it too).
+        if (j > 0) {
+          if (!(ok = mbar_wait_warp(&bar.ot_full[ti], (j - 1) & 1))) break;
+          tc_fence_after();
+        }
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int c = 0; c < DH; c += 32) {
+            tmem_ld32(tO + c, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 o = fmul2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])),
+                                     make_float2(alpha, alpha));
+              x[e] = __float_as_uint(o.x);
+              x[e + 1] = __float_as_uint(o.y);
+            }
+            tmem_st32(tO + c, x);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.o_ready[ti]);
+      }
+    }
+    // ---- epilogue: out = O / l * delta_V on this half's columns (l carries the 448)
+    if (nTi[ti] > 0) {
+      float* lb = s_l + ti * 256;
+      lb[hf * 128 + row] = l;
+      __syncwarp();
+      uint64_t* lxbar = bar.lx + ti * 4 + quarter;
+      if (lane == 0) mbar_arrive(lxbar);
+      if (ok) ok = mbar_wait_warp(lxbar, 0);
+      l += lb[(1 - hf) * 128 + row];
+      // TMEM accumulator: the last P V must have retired (two-level: this warp
+      // already formed the final sum)
+      if (ok && !TWO_LEVEL) ok = mbar_wait_warp(&bar.ot_full[ti], (nTi[ti] - 1) & 1);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l;
+        if (LSE && hf == 0 && qrow < a.N) {
+          // ln sum_j e^(S_ij) = (m + log2(l / 448)) ln 2 (m: running max of the
+          // log2-domain scores, l: sum of 448 2^(t - m)), plus the smooth-K shift
+          const int64_t bhq64 = (int64_t)(b * a.Hq + h);
+          a.lse[bhq64 * a.N + qrow] =
+              l > 0.0f ? (m + log2f(l) - kLog2_448) * 0.69314718055994531f + a.sm_scale * a.qkm[bhq64 * a.Np + qrow]
+                       : -INFINITY;
+        }
+        const float* sv = a.s_v + (int64_t)(b * a.Hkv + g) * D + DH * hf;
+        // row qrow of head (b, h): one formula for either layout (strides from the host)
+        TO* out = reinterpret_cast<TO*>(a.o) + b * a.o_bs + h * a.o_hs + qrow * a.o_rs + DH * hf;
+#pragma unroll
+        for (int c = 0; c < DH; c += 32) {
+          tmem_ld32(tO + c, x);
+          tmem_ld_wait();
+          if (qrow < a.N) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              float f[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(x[e + u]) * inv_l * __ldg(sv + c + e + u);
+              *reinterpret_cast<uint4*>(out + c + e) = make_uint4(pack2<TO>(f[0], f[1]), pack2<TO>(f[2], f[3]),
+                                                                  pack2<TO>(f[4], f[5]), pack2<TO>(f[6], f[7]));
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Bit-exactness probe: one INT32 tile Q^_i K^_j^T through the same TMA layout,
 // descriptors and kind::i8 instruction as the attention kernel.
 template <int D>
@@ -852,14 +1419,17 @@ __global__ void bounded_wait_probe_kernel() {
 template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO>
 cudaError_t launch_attn_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                           cudaStream_t st) {
-  auto kern = a.lse ? attn_i8f8_kernel<D, CAUSAL, HAS_DS, TWO_LEVEL, TO, true>
-                    : attn_i8f8_kernel<D, CAUSAL, HAS_DS, TWO_LEVEL, TO, false>;
-  const int smem = (int)Smem<D>::kBytes;
+  // with delta_S the split-row kernel, else the one-warp-per-row kernel
+  auto kern = HAS_DS ? (a.lse ? attn_i8f8_split_kernel<D, CAUSAL, true, TWO_LEVEL, TO, true>
+                              : attn_i8f8_split_kernel<D, CAUSAL, true, TWO_LEVEL, TO, false>)
+                     : (a.lse ? attn_i8f8_kernel<D, CAUSAL, false, TWO_LEVEL, TO, true>
+                              : attn_i8f8_kernel<D, CAUSAL, false, TWO_LEVEL, TO, false>);
+  const int smem = HAS_DS ? (int)SmemSplit<D>::kBytes : (int)Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned n_pairs = (unsigned)(a.n_qtiles + 1) / 2;
   const unsigned grid = n_pairs * (unsigned)(a.B * a.Hq);
-  kern<<<grid, kThreadsAttn, smem, st>>>(tmQ, tmK, tmV, a);
+  kern<<<grid, HAS_DS ? kThreadsSplit : kThreadsAttn, smem, st>>>(tmQ, tmK, tmV, a);
   return cudaGetLastError();
 }
 
