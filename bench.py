@@ -39,16 +39,24 @@ FP4_PER_BF16 = 4.0  # nominal dense ratio 9 / 2.25 PFLOP/s
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch of the prefill workload: one ncu capture of attn_i8f8_kernel at B=3
-# (482.4 MB), scaled to B=4 by the number of heads.  Valid only for the kernel
-# source it was taken on (hash below); any other source reports null.
-ATTN_TRAFFIC = {"bytes": 482.4e6 * 4 / 3, "src_sha256_16": "7059f06be6cfa67e", "workload": "llm_prefill_causal_B4_H32_N4096_d128"}
+# (418.0 + 67.4 MB), scaled to B=4 by the number of heads.  Valid only for the
+# kernel sources it was taken on (hash below); any other source reports null.
+ATTN_TRAFFIC = {"bytes": (418020608 + 67446784) * 4 / 3, "src_sha256_16": "106106c1f65b8b92",
+                "workload": "llm_prefill_causal_B4_H32_N4096_d128"}
+
+
+def _attn_src_sha() -> str:
+    """Hash of the sources that decide the attention kernel's memory traffic."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("attn_i8f8.cu", "common.cuh"):
+        with open(os.path.join(_ROOT, "quantized_attention_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def _attn_traffic(w: W.Workload):
-    import hashlib
-    src = os.path.join(_ROOT, "quantized_attention_block_b200", "csrc", "attn_i8f8.cu")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    sha = _attn_src_sha()
     if sha != ATTN_TRAFFIC["src_sha256_16"] or w.name != ATTN_TRAFFIC["workload"]:
         return None
     return ATTN_TRAFFIC["bytes"]
@@ -121,6 +129,11 @@ class ClockSampler:
             if len(first) != 2 or first[0] != "max":
                 raise RuntimeError("sampler did not start: " + self.proc.stderr.read()[-300:])
             self.max_sm = int(first[1])
+            # one sample before the caller's region starts (a short region may
+            # otherwise end before the first sample)
+            f = self.proc.stdout.readline().split()
+            if len(f) == 4:
+                self.samples.append((int(f[0]), int(f[1]), int(f[2]), float(f[3])))
         except Exception as e:  # pragma: no cover
             self.err = f"nvml unavailable: {e}"
             self.proc = None

@@ -230,8 +230,8 @@ def _sample_tiles(n_tiles, rng, k=3):
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_quant_bit_exact_and_sampled_attention(name, mode):
     """At the benchmark's sizes and launch configuration: every quantised value
-    checked bit-exactly; attention outputs on sampled Q tiles of sampled heads
-    (first, last / ragged tail, random) checked element by element."""
+    checked bit-exactly; attention outputs on sampled Q tiles of five sampled
+    heads (first, last / ragged tail, random) checked element by element."""
     w = W.get(name)
     q, k, v = W.make_qkv(w)
     p, ws, view, o = gpu_attention(w, q, k, v, PV_MODES[mode])
@@ -240,7 +240,13 @@ def test_full_size_quant_bit_exact_and_sampled_attention(name, mode):
     assert not bad, bad
     rng = np.random.default_rng(123)
     n_tiles = int(view.Np) // 128
-    heads = sorted({(0, 0), (w.B - 1, w.Hq - 1), (int(rng.integers(0, w.B)), int(rng.integers(0, w.Hq)))})
+    # five (batch, head) pairs (the first, the last, three at random: for GQA
+    # they span several KV groups) x four Q tiles (first, last / ragged, two at
+    # random): about 20 tiles per workload
+    heads = {(0, 0), (w.B - 1, w.Hq - 1)}
+    while len(heads) < min(5, w.B * w.Hq):
+        heads.add((int(rng.integers(0, w.B)), int(rng.integers(0, w.Hq))))
+    heads = sorted(heads)
     from concurrent.futures import ThreadPoolExecutor
     jobs = []
     for (b, h) in heads:
