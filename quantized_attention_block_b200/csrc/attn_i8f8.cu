@@ -510,9 +510,49 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       if (lane == 0) mbar_arrive(&bar.p_full[ti * 2 + (j & 1)]);
       l = fmaf(l, alpha, rs2.x + rs2.y);
       m = m_new;
+      if constexpr (TWO_LEVEL) {
+        // Level 2 in this warpgroup, whose registers can hold a whole O_t row:
+        // P V(j) put a fresh O_t into S_i's columns [0, D).  Read it (S is dead),
+        // give S_i's columns their magic fill back and let the next Q K^T run,
+        // then form O = alpha O + O_t while that MMA works.
+        if (!(ok = mbar_wait_warp(&bar.ot_full[ti], j & 1))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D; c += 32) tmem_ld32p(tS + c, s + c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) tmem_fill8(tS + c, kMagicBits);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.r_free[ti]);
+        const uint32_t tO = tmem + 256 + D * ti + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t x[32];
+          if (j == 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = s[c + e];
+          } else {
+            tmem_ld32(tO + c, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 o = ffma2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])),
+                                     make_float2(alpha, alpha),
+                                     make_float2(__uint_as_float(s[c + e]), __uint_as_float(s[c + e + 1])));
+              x[e] = __float_as_uint(o.x);
+              x[e + 1] = __float_as_uint(o.y);
+            }
+          }
+          tmem_st32(tO + c, x);
+        }
+        tmem_st_wait();  // O is final before l_ready (the epilogue reads it)
+      }
     }
     s_l[ti * 128 + row] = l;
     if (LSE) s_l[256 + ti * 128 + row] = m;
+    tc_fence_before();  // (two-level) this warp's O stores before the epilogue's reads
     mbar_arrive(&bar.l_ready[ti]);
   } else {
     // ------------------------------------------------------------ correction + epilogue
@@ -521,67 +561,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
-    uint32_t x[32], y[32];
+    uint32_t x[32];
     // every phase of p_full[tile][buffer] is waited in order, j = 0 included (a
-    // parity wait on a phase two ahead of the barrier would pass at once)
+    // parity wait on a phase two ahead of the barrier would pass at once).
+    // Two-level mode: the softmax warpgroups form the level-2 sums themselves;
+    // this warpgroup only writes the output.
     if constexpr (TWO_LEVEL) {
-      for (int j = 0; j < nT && ok; ++j) {
-        for (int i = 0; i < 2; ++i) {
-          if (j >= nTi[i]) continue;
-          if (!(ok = mbar_wait_warp(&bar.ot_full[i], j & 1))) break;
-          if (!(ok = mbar_wait_warp(&bar.p_full[i * 2 + (j & 1)], (j >> 1) & 1))) break;
-          tc_fence_after();
-          const float alpha = s_alpha[(i * 2 + (j & 1)) * 128 + row];
-          const uint32_t tOt = tmem + 128 * i + lane_off, tO = tmem + 256 + D * i + lane_off;
-          if (j == 0) {
-  #pragma unroll
-            for (int c = 0; c < D; c += 32) {
-              tmem_ld32(tOt + c, x);
-              tmem_ld_wait();
-              tmem_st32(tO + c, x);
-            }
-          } else {
-            // O = alpha * O + O_t in 16-column chunks; the loads of chunk c + 1
-            // are in flight while chunk c is combined and stored.
-            uint32_t* xa = x;
-            uint32_t* ya = y;
-            uint32_t* xb = x + 16;
-            uint32_t* yb = y + 16;
-            tmem_ld16p(tOt, xa);
-            tmem_ld16p(tO, ya);
-            tmem_ld_wait();
-  #pragma unroll
-            for (int c = 0; c < D; c += 16) {
-              uint32_t* xc = (c / 16) % 2 == 0 ? xa : xb;
-              uint32_t* yc = (c / 16) % 2 == 0 ? ya : yb;
-              uint32_t* xn = (c / 16) % 2 == 0 ? xb : xa;
-              uint32_t* yn = (c / 16) % 2 == 0 ? yb : ya;
-              if (c + 16 < D) {
-                tmem_ld16p(tOt + c + 16, xn);
-                tmem_ld16p(tO + c + 16, yn);
-              }
-  #pragma unroll
-              for (int e = 0; e < 16; e += 2) {
-                const float2 o = ffma2(make_float2(__uint_as_float(yc[e]), __uint_as_float(yc[e + 1])),
-                                       make_float2(alpha, alpha),
-                                       make_float2(__uint_as_float(xc[e]), __uint_as_float(xc[e + 1])));
-                xc[e] = __float_as_uint(o.x);
-                xc[e + 1] = __float_as_uint(o.y);
-              }
-              tmem_st16p(tO + c, xc);
-              if (c + 16 < D) tmem_ld_wait();
-            }
-          }
-          // S_i's columns get the magic fill back (O_t covered the first D of them;
-          // the softmax read all 128 before P V(j) could run)
-  #pragma unroll
-          for (int c = 0; c < 128; c += 8) tmem_fill8(tOt + c, kMagicBits);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar.r_free[i]);
-        }
-      }
     } else {
       // O_i accumulates in TMEM; before PV(i, j) adds tile j, rows whose max grew
       // are rescaled by alpha = e^(m_old - m_new).  A warp whose 32 rows all have
