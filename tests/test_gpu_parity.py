@@ -36,6 +36,11 @@ EDGE = {
     "N385_bq32_smoothq_d64": W.get("video").with_(name="N385_bq32", B=1, Hq=2, Hkv=2, N=385, bq=32),
     "N260_bq32_smoothq_gqa_causal": W.get("gqa").with_(name="N260_bq32_sq", B=1, Hq=4, Hkv=2, N=260, bq=32,
                                                         smooth_q=True, qk_shared_bias_std=0.0, k_bias_std=3.0),
+    # delta_S cases for the split-row kernel: fp16 at d = 64, non-causal d = 128
+    "N333_fp16_smoothq_d64": W.get("video").with_(name="N333_fp16_sq", B=1, Hq=2, Hkv=2, N=333,
+                                                  dtype=torch.float16),
+    "N450_smoothq_d128": W.get("prefill").with_(name="N450_sq", B=1, Hq=2, Hkv=2, N=450, causal=False,
+                                                smooth_q=True, qk_shared_bias_std=2.0),
 }
 
 
