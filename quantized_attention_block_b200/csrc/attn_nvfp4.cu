@@ -345,16 +345,14 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
             ++released;
           }
           if (next_pv[0] >= nTi[0] && next_pv[1] >= nTi[1] && released >= nT) break;
+          // spin (a sleep here delays the reaction to a ready operand), bounded by the idle time
           if (progress) {
             t_idle = 0;
           } else if (t_idle == 0) {
-            __nanosleep(32);
             t_idle = globaltimer_ns();
           } else if (globaltimer_ns() - t_idle > g_wait_limit_ns) {
             record_error(kDevErrTimeout);
             ok = false;
-          } else {
-            __nanosleep(32);
           }
         }
         mma_commit(bar.mma_done);
