@@ -84,7 +84,8 @@ struct Smem {
   static constexpr uint32_t oDS = oP + 4 * kP;           // kStages
   static constexpr uint32_t oAlpha = oDS + kStages * kDS;  // float[tile][buffer][128]
   static constexpr uint32_t oL = oAlpha + 4 * 128 * 4;   // float[2][128] l, then float[2][128] m
-  static constexpr uint32_t oBar = oL + 2 * 2 * 128 * 4;
+  static constexpr uint32_t oSV = oL + 2 * 2 * 128 * 4;  // float[D] delta_V of the KV head (epilogue)
+  static constexpr uint32_t oBar = oSV + D * 4;
   static constexpr uint32_t kNumBars = 1 + 3 * kStages + 2 + 4 + 4 + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t oTmem = oBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = oTmem + 16 + 1024;  // + alignment slack
@@ -562,6 +563,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
     uint32_t x[32];
+    // delta_V of this KV head into shared memory now, while the tile loop
+    // runs: read from global in the epilogue, its first touch of each line
+    // would miss L1 once per 32-column chunk
+    float* s_sv = reinterpret_cast<float*>(smem + L::oSV);
+    if (row < D) s_sv[row] = __ldg(a.s_v + (int64_t)(b * a.Hkv + g) * D + row);
+    named_bar_sync(1, 128);
     // every phase of p_full[tile][buffer] is waited in order, j = 0 included (a
     // parity wait on a phase two ahead of the barrier would pass at once).
     // Two-level mode: the softmax warpgroups form the level-2 sums themselves;
@@ -619,7 +626,6 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             l > 0.0f ? (m + log2f(l) - kLog2_448) * 0.69314718055994531f + a.sm_scale * a.qkm[bhq * a.Np + qrow]
                      : -INFINITY;
       }
-      const float* sv = a.s_v + (int64_t)(b * a.Hkv + g) * D;
       // row qrow of head (b, h): one formula for either layout (strides from the host)
       TO* out = reinterpret_cast<TO*>(a.o) + b * a.o_bs + h * a.o_hs + qrow * a.o_rs;
       const uint32_t tO = tmem + 256 + D * i + lane_off;
@@ -632,7 +638,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           for (int e = 0; e < 32; e += 8) {
             float f[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(x[e + u]) * inv_l * __ldg(sv + c + e + u);
+            for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(x[e + u]) * inv_l * s_sv[c + e + u];
             *reinterpret_cast<uint4*>(out + c + e) =
                 make_uint4(pack2<TO>(f[0], f[1]), pack2<TO>(f[2], f[3]), pack2<TO>(f[4], f[5]), pack2<TO>(f[6], f[7]));
           }

@@ -25,6 +25,13 @@ __device__ __forceinline__ void record_error(unsigned int code) {
 
 // An error recorded by an earlier kernel (e.g. a quantiser's wait that ran out)
 // and not yet read by the host.
+// Barrier `id` (1..15) over `threads` threads (a multiple of 32) of the CTA:
+// every warp of the group must reach it (no timeout: use it only where every
+// participating warp arrives unconditionally)
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ bool device_error_pending() {
   return *reinterpret_cast<volatile unsigned int*>(&g_device_error) != 0u;
 }
