@@ -161,14 +161,6 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   bar.mma_done = bar.o_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oTmem);
 
-  // An unread device error (a quantiser wait that ran out leaves some codes
-  // unwritten) stops the launch before it reads the quantised tensors: O is
-  // left as it was rather than computed from stale codes.
-  __shared__ int s_skip;
-  if (threadIdx.x == 0) s_skip = device_error_pending() ? 1 : 0;
-  __syncthreads();
-  if (s_skip) return;
-
   // ---- work: (b, h, pair of Q tiles), heavy causal pairs first
   const int bhq = a.B * a.Hq;
   const int n_pairs = (a.n_qtiles + 1) / 2;
@@ -187,7 +179,37 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int wg = warp / 4;
+  // TMA loads of K_j (with the delta_S rows of both Q tiles) and V_j^T into
+  // ring stage j % kStages; krow0 / vrow: the KV head's first K row and V^T row
+  auto issue_kv = [&](int j, int krow0, int vrow) {
+    const int s = j % kStages;
+    const int ds_rows = kTile / a.bq;  // Q blocks per tile (1, 2 or 4)
+    const uint32_t ds_bytes = (uint32_t)((nTi[0] > 0) + (nTi[1] > 0)) * ds_rows * 512;
+    mbar_expect_tx(&bar.k_full[s], L::kK + (HAS_DS ? ds_bytes : 0u));
+    tma_load_2d(sK + s * L::kK, &tmK, &bar.k_full[s], 0, krow0 + j * kTile);
+    if (HAS_DS) {
+      // delta_S[b, h, Q block, keys of tile j] for the Q blocks of both tiles
+      for (int i = 0; i < 2; ++i)
+        for (int hb = 0; hb < ds_rows; ++hb)
+          if (nTi[i] > 0) {
+            const int blk = min((2 * pr + i) * ds_rows + hb, a.Tm - 1);
+            bulk_load_1d(smem + L::oDS + s * L::kDS + (i * 4 + hb) * 512,
+                         a.dS + ((int64_t)(b * a.Hq + h) * a.Tm + blk) * a.Np + (int64_t)j * kTile, 512,
+                         &bar.k_full[s]);
+          }
+    }
+    mbar_expect_tx(&bar.v_full[s], L::kV);
+    tma_load_2d(sV + s * L::kV, &tmV, &bar.v_full[s], j * kTile, vrow);
+  };
+  // Thread 0 initialises the barriers and, before the CTA's first barrier,
+  // starts the loads of both Q tiles and of the first kStages K / V tiles, so
+  // that their latency overlaps the TMEM allocation and the magic fill.  An
+  // unread device error (a quantiser wait that ran out leaves some codes
+  // unwritten) stops the launch before anything reads the quantised tensors:
+  // O is left as it was rather than computed from stale codes.
+  __shared__ int s_skip;
   if (threadIdx.x == 0) {
+    const bool pending = device_error_pending();
     mbar_init(bar.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar.k_full[s], 1);
@@ -207,6 +229,18 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
     mbar_init(bar.mma_done, 1);
     mbar_fence_init();
+    s_skip = pending ? 1 : 0;
+    if (!pending) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+      const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
+      mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
+      for (int i = 0; i < 2; ++i)
+        if (nTi[i] > 0) tma_load_2d(sQ + i * L::kQ, &tmQ, bar.q_full, 0, (int)(qhead + (int64_t)(2 * pr + i) * kTile));
+      const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np), vrow = (b * a.Hkv + g) * D;
+      for (int j = 0; j < nT && j < kStages; ++j) issue_kv(j, krow0, vrow);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -215,6 +249,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (s_skip) {
+    if (warp == 1) tmem_dealloc(*tmem_slot, kTmemCols);
+    return;
+  }
   const uint32_t tmem = *tmem_slot;
   // S accumulators start at the int32 bit pattern of 1.5 * 2^23: QK^T accumulates
   // onto it, so TMEM returns 0x4B400000 + acc, which read as fp32 is exactly
@@ -233,38 +271,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     regs_dec<kRegsProducer>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
-      tma_prefetch_map(&tmQ);
-      tma_prefetch_map(&tmK);
-      tma_prefetch_map(&tmV);
-      const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
-      const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np);
-      const int vrow = (b * a.Hkv + g) * D;
-      const int ds_rows = kTile / a.bq;  // Q blocks per tile (1, 2 or 4)
-      const uint32_t ds_bytes = (uint32_t)((nTi[0] > 0) + (nTi[1] > 0)) * ds_rows * 512;
-      mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
-      for (int i = 0; i < 2; ++i)
-        if (nTi[i] > 0) tma_load_2d(sQ + i * L::kQ, &tmQ, bar.q_full, 0, (int)(qhead + (int64_t)(2 * pr + i) * kTile));
+      // (Q and K / V tiles 0 .. kStages - 1 went out before the first barrier)
+      const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np), vrow = (b * a.Hkv + g) * D;
       bool ok = true;
-      int j = 0;
+      int j = nT < kStages ? nT : kStages;
       for (; j < nT && ok; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages) ok = mbar_wait(&bar.kv_empty[s], ((j / kStages) + 1) & 1);
-        if (!ok) break;
-        mbar_expect_tx(&bar.k_full[s], L::kK + (HAS_DS ? ds_bytes : 0u));
-        tma_load_2d(sK + s * L::kK, &tmK, &bar.k_full[s], 0, krow0 + j * kTile);
-        if (HAS_DS) {
-          // delta_S[b, h, Q block, keys of tile j] for the Q blocks of both tiles
-          for (int i = 0; i < 2; ++i)
-            for (int hb = 0; hb < ds_rows; ++hb)
-              if (nTi[i] > 0) {
-                const int blk = min((2 * pr + i) * ds_rows + hb, a.Tm - 1);
-                bulk_load_1d(smem + L::oDS + s * L::kDS + (i * 4 + hb) * 512,
-                             a.dS + ((int64_t)(b * a.Hq + h) * a.Tm + blk) * a.Np + (int64_t)j * kTile, 512,
-                             &bar.k_full[s]);
-              }
-        }
-        mbar_expect_tx(&bar.v_full[s], L::kV);
-        tma_load_2d(sV + s * L::kV, &tmV, &bar.v_full[s], j * kTile, vrow);
+        if (!(ok = mbar_wait(&bar.kv_empty[j % kStages], ((j / kStages) + 1) & 1))) break;
+        issue_kv(j, krow0, vrow);
       }
       // never leave a copy in flight
       for (int jj = (j - kStages > 0 ? j - kStages : 0); jj < j; ++jj) {
