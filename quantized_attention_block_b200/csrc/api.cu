@@ -150,6 +150,20 @@ bool map_input(CUtensorMap* m, const void* base, uint64_t D, uint64_t N, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The caller's 16-bit output as a TMA tensor for bulk stores: 4D (d, N, Hq, B)
+// with the strides of either layout, box 64 columns x 32 rows, 128-byte swizzle.
+bool map_output(CUtensorMap* m, void* base, const AttnArgs& a) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)a.D, (cuuint64_t)a.N, (cuuint64_t)a.Hq, (cuuint64_t)a.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)a.o_rs * 2, (cuuint64_t)a.o_hs * 2, (cuuint64_t)a.o_bs * 2};
+  const cuuint32_t box[4] = {64, 32, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 sage_status fill_view(const sage_params* p, const Dims& d, void* ws, sage_quant_view* v) {
   const Layout L = make_layout(p, d);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -400,7 +414,9 @@ sage_status sage_attn_fwd_quantized_lse(const sage_quant_view* view, void* o, fl
   AttnArgs a = attn_args(view, p, d);
   a.o = o;
   a.lse = lse;
-  return from_cuda(launch_attn_i8f8(a, mQ, mK, mV, static_cast<cudaStream_t>(stream)));
+  CUtensorMap mO;
+  if (!map_output(&mO, o, a)) return SAGE_ERR_CUDA;
+  return from_cuda(launch_attn_i8f8(a, mQ, mK, mV, mO, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* o, const sage_params* p,

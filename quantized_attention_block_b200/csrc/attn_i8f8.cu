@@ -128,7 +128,8 @@ struct Bars {
 template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO, bool LSE>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const AttnArgs a) {
   using L = Smem<D>;
   constexpr uint32_t kSwzQK = (D == 128) ? kSwizzle128B : kSwizzle64B;
   constexpr uint32_t kSboQK = 8 * D;  // 8 rows x D bytes per swizzle atom
@@ -639,25 +640,39 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             l > 0.0f ? (m + log2f(l) - kLog2_448) * 0.69314718055994531f + a.sm_scale * a.qkm[bhq * a.Np + qrow]
                      : -INFINITY;
       }
-      // row qrow of head (b, h): one formula for either layout (strides from the host)
-      TO* out = reinterpret_cast<TO*>(a.o) + b * a.o_bs + h * a.o_hs + qrow * a.o_rs;
+      // The warp stages its 32 output rows in tile i's P buffers (free: the
+      // tile's last P V retired) as boxes of 64 columns x 32 rows in the TMA
+      // 128-byte swizzle (16-byte chunk q of row r at q ^ (r & 7)), and one lane
+      // writes them out with bulk tensor stores (rows past N are clipped by the
+      // tensor map): no per-thread global stores.
+      constexpr int kBoxes = D * (int)sizeof(TO) / 128;  // 64-column boxes per row (1 or 2)
+      uint8_t* stg = sP + i * 2 * L::kP + quarter * kBoxes * 4096;
       const uint32_t tO = tmem + 256 + D * i + lane_off;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         tmem_ld32(tO + c, x);
         tmem_ld_wait();
-        if (qrow < a.N) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            float f[8];
+        for (int e = 0; e < 32; e += 8) {
+          float f[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(x[e + u]) * inv_l * s_sv[c + e + u];
-            *reinterpret_cast<uint4*>(out + c + e) =
-                make_uint4(pack2<TO>(f[0], f[1]), pack2<TO>(f[2], f[3]), pack2<TO>(f[4], f[5]), pack2<TO>(f[6], f[7]));
-          }
+          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(x[e + u]) * inv_l * s_sv[c + e + u];
+          const int col = c + e, q = (col % 64) / 8;
+          *reinterpret_cast<uint4*>(stg + (col / 64) * 4096 + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+              make_uint4(pack2<TO>(f[0], f[1]), pack2<TO>(f[2], f[3]), pack2<TO>(f[4], f[5]), pack2<TO>(f[6], f[7]));
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int qrow0 = (2 * pr + i) * kTile + quarter * 32;
+      if (lane == 0 && qrow0 < a.N) {
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) tma_store_4d(&tmO, stg + bx * 4096, bx * 64, qrow0, h, b);
+        bulk_commit();
+      }
     }
+    // the bulk stores have read their shared-memory source before the CTA ends
+    if (lane == 0) bulk_wait_read_all();
   }
 
   // ---------------------------------------------------------------- teardown
@@ -735,7 +750,8 @@ struct BarsSplit {
 template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO, bool LSE>
 __global__ void __launch_bounds__(kThreadsSplit, 1)
     attn_i8f8_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+                     const __grid_constant__ CUtensorMap tmV,
+                           const __grid_constant__ CUtensorMap /*tmO: unused*/, const AttnArgs a) {
   using L = SmemSplit<D>;
   constexpr uint32_t kSwzQK = (D == 128) ? kSwizzle128B : kSwizzle64B;
   constexpr uint32_t kSboQK = 8 * D;  // 8 rows x D bytes per swizzle atom
@@ -1422,7 +1438,7 @@ __global__ void bounded_wait_probe_kernel() {
 
 template <int D, bool CAUSAL, bool HAS_DS, bool TWO_LEVEL, typename TO>
 cudaError_t launch_attn_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                          cudaStream_t st) {
+                          const CUtensorMap& tmO, cudaStream_t st) {
   // with delta_S the split-row kernel, else the one-warp-per-row kernel
   auto kern = HAS_DS ? (a.lse ? attn_i8f8_split_kernel<D, CAUSAL, true, TWO_LEVEL, TO, true>
                               : attn_i8f8_split_kernel<D, CAUSAL, true, TWO_LEVEL, TO, false>)
@@ -1433,34 +1449,37 @@ cudaError_t launch_attn_t(const AttnArgs& a, const CUtensorMap& tmQ, const CUten
   if (e != cudaSuccess) return e;
   const unsigned n_pairs = (unsigned)(a.n_qtiles + 1) / 2;
   const unsigned grid = n_pairs * (unsigned)(a.B * a.Hq);
-  kern<<<grid, HAS_DS ? kThreadsSplit : kThreadsAttn, smem, st>>>(tmQ, tmK, tmV, a);
+  kern<<<grid, HAS_DS ? kThreadsSplit : kThreadsAttn, smem, st>>>(tmQ, tmK, tmV, tmO, a);
   return cudaGetLastError();
 }
 
 template <int D, bool CAUSAL, bool TWO_LEVEL>
 cudaError_t launch_attn_m(const AttnArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                          cudaStream_t st) {
+                          const CUtensorMap& o, cudaStream_t st) {
   if (a.dS) {
-    return a.out_fp16 ? launch_attn_t<D, CAUSAL, true, TWO_LEVEL, __half>(a, q, k, v, st)
-                      : launch_attn_t<D, CAUSAL, true, TWO_LEVEL, __nv_bfloat16>(a, q, k, v, st);
+    return a.out_fp16 ? launch_attn_t<D, CAUSAL, true, TWO_LEVEL, __half>(a, q, k, v, o, st)
+                      : launch_attn_t<D, CAUSAL, true, TWO_LEVEL, __nv_bfloat16>(a, q, k, v, o, st);
   }
-  return a.out_fp16 ? launch_attn_t<D, CAUSAL, false, TWO_LEVEL, __half>(a, q, k, v, st)
-                    : launch_attn_t<D, CAUSAL, false, TWO_LEVEL, __nv_bfloat16>(a, q, k, v, st);
+  return a.out_fp16 ? launch_attn_t<D, CAUSAL, false, TWO_LEVEL, __half>(a, q, k, v, o, st)
+                    : launch_attn_t<D, CAUSAL, false, TWO_LEVEL, __nv_bfloat16>(a, q, k, v, o, st);
 }
 
 template <int D, bool CAUSAL>
 cudaError_t launch_attn_d(const AttnArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                          cudaStream_t st) {
-  return a.two_level ? launch_attn_m<D, CAUSAL, true>(a, q, k, v, st) : launch_attn_m<D, CAUSAL, false>(a, q, k, v, st);
+                          const CUtensorMap& o, cudaStream_t st) {
+  return a.two_level ? launch_attn_m<D, CAUSAL, true>(a, q, k, v, o, st)
+                     : launch_attn_m<D, CAUSAL, false>(a, q, k, v, o, st);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                             const CUtensorMap& tmV, cudaStream_t st) {
+                             const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t st) {
   if (a.D == 128)
-    return a.causal ? launch_attn_d<128, true>(a, tmQ, tmK, tmV, st) : launch_attn_d<128, false>(a, tmQ, tmK, tmV, st);
-  return a.causal ? launch_attn_d<64, true>(a, tmQ, tmK, tmV, st) : launch_attn_d<64, false>(a, tmQ, tmK, tmV, st);
+    return a.causal ? launch_attn_d<128, true>(a, tmQ, tmK, tmV, tmO, st)
+                    : launch_attn_d<128, false>(a, tmQ, tmK, tmV, tmO, st);
+  return a.causal ? launch_attn_d<64, true>(a, tmQ, tmK, tmV, tmO, st)
+                  : launch_attn_d<64, false>(a, tmQ, tmK, tmV, tmO, st);
 }
 
 cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, cudaStream_t st) {

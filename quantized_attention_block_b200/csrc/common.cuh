@@ -100,8 +100,10 @@ struct QuantMaps {
 // else the two-pass path)
 int quant_kernel_count(const QuantArgs& a, int is_fp16, bool allow_one_read);
 cudaError_t launch_quant(const QuantArgs& a, const QuantMaps& m, int is_fp16, cudaStream_t st);
+// tmO: the caller's output as a 4D tensor (d, N, Hq, B), box 64 x 32, 128-byte
+// swizzle (the one-warp-per-row kernel writes its output tiles through it)
 cudaError_t launch_attn_i8f8(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                             const CUtensorMap& tmV, cudaStream_t st);
+                             const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t st);
 cudaError_t launch_qk_probe(const AttnArgs& a, const CUtensorMap& tmQ, const CUtensorMap& tmK, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(cudaStream_t st);
 cudaError_t launch_exp2_poly_probe(const float* x, float* y, int n, cudaStream_t st);
