@@ -206,11 +206,15 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   // starts the loads of both Q tiles and of the first kStages K / V tiles, so
   // that their latency overlaps the TMEM allocation and the magic fill.  An
   // unread device error (a quantiser wait that ran out leaves some codes
-  // unwritten) stops the launch before anything reads the quantised tensors:
-  // O is left as it was rather than computed from stale codes.
+  // unwritten) stops the launch before anything is computed from the
+  // quantised tensors: O is left as it was rather than computed from stale
+  // codes.  The error word is read first but looked at only after the loads
+  // are out, so its latency is off their path; with an error pending the CTA
+  // lets those loads land and ends.
   __shared__ int s_skip;
   if (threadIdx.x == 0) {
-    const bool pending = device_error_pending();
+    const int pending = device_error_pending() ? 1 : 0;
+    const int j_pre = nT < kStages ? nT : kStages;  // K / V tiles loaded before the first barrier
     mbar_init(bar.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar.k_full[s], 1);
@@ -230,17 +234,23 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
     mbar_init(bar.mma_done, 1);
     mbar_fence_init();
-    s_skip = pending ? 1 : 0;
-    if (!pending) {
-      tma_prefetch_map(&tmQ);
-      tma_prefetch_map(&tmK);
-      tma_prefetch_map(&tmV);
-      const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
-      mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
-      for (int i = 0; i < 2; ++i)
-        if (nTi[i] > 0) tma_load_2d(sQ + i * L::kQ, &tmQ, bar.q_full, 0, (int)(qhead + (int64_t)(2 * pr + i) * kTile));
-      const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np), vrow = (b * a.Hkv + g) * D;
-      for (int j = 0; j < nT && j < kStages; ++j) issue_kv(j, krow0, vrow);
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmV);
+    const int64_t qhead = (int64_t)(b * a.Hq + h) * a.Np;
+    mbar_expect_tx(bar.q_full, (nTi[0] > 0 ? L::kQ : 0u) + (nTi[1] > 0 ? L::kQ : 0u));
+    for (int i = 0; i < 2; ++i)
+      if (nTi[i] > 0) tma_load_2d(sQ + i * L::kQ, &tmQ, bar.q_full, 0, (int)(qhead + (int64_t)(2 * pr + i) * kTile));
+    const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np), vrow = (b * a.Hkv + g) * D;
+    for (int j = 0; j < j_pre; ++j) issue_kv(j, krow0, vrow);
+    s_skip = pending;
+    if (pending) {
+      // never leave a copy in flight (bounded waits)
+      mbar_wait(bar.q_full, 0);
+      for (int j = 0; j < j_pre; ++j) {
+        mbar_wait(&bar.k_full[j], 0);
+        mbar_wait(&bar.v_full[j], 0);
+      }
     }
   }
   if (warp == 1) {
@@ -275,7 +285,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       // (Q and K / V tiles 0 .. kStages - 1 went out before the first barrier)
       const int krow0 = (int)((int64_t)(b * a.Hkv + g) * a.Np), vrow = (b * a.Hkv + g) * D;
       bool ok = true;
-      int j = nT < kStages ? nT : kStages;
+      int j = nT < kStages ? nT : kStages;  // (tiles below went out before the first barrier)
       for (; j < nT && ok; ++j) {
         if (!(ok = mbar_wait(&bar.kv_empty[j % kStages], ((j / kStages) + 1) & 1))) break;
         issue_kv(j, krow0, vrow);
