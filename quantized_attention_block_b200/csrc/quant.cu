@@ -99,10 +99,12 @@ __device__ __forceinline__ uint2 quant8_i8(const float (&x)[8], float s, float r
 }
 
 // Two E4M3 codes of x0 / s, x1 / s (lo byte x0); s > 0, r = RN(1/s).
+// (the products run as f32x2 pairs: each lane is the same IEEE RN product)
 __device__ __forceinline__ uint32_t quant_e4m3x2(float x0, float x1, float s, float r) {
-  const float y0 = __fmul_rn(x0, r), y1 = __fmul_rn(x1, r);
-  const uint32_t lo = cvt_e4m3x2(__fmul_rn(y0, kBracketLo), __fmul_rn(y1, kBracketLo));
-  const uint32_t hi = cvt_e4m3x2(__fmul_rn(y0, kBracketHi), __fmul_rn(y1, kBracketHi));
+  const float2 y = fmul2(make_float2(x0, x1), make_float2(r, r));
+  const float2 yl = fmul2(y, make_float2(kBracketLo, kBracketLo));
+  const float2 yh = fmul2(y, make_float2(kBracketHi, kBracketHi));
+  const uint32_t lo = cvt_e4m3x2(yl.x, yl.y), hi = cvt_e4m3x2(yh.x, yh.y);
   return lo == hi ? lo : cvt_e4m3x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
 }
 
