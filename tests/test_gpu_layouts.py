@@ -60,3 +60,31 @@ def test_nhd_equals_hnd_nvfp4(two_pass):
         sage.sage_debug_kv_quant_two_pass(False)
     assert sage.sage_last_device_error() == 0
     assert torch.equal(o_n.transpose(1, 2).contiguous().view(torch.int16), o_h.view(torch.int16))
+
+
+@pytest.mark.parametrize("layout", ["HND", "NHD"])
+@pytest.mark.parametrize("pv_accum", [sage.PV_TWO_LEVEL, sage.PV_TMEM_FP32])
+def test_output_writes_stay_inside_o(layout, pv_accum):
+    """The output tiles leave the kernel by bulk tensor stores whose map clips
+    rows past N: with a ragged N (the last Q tile is mostly past N) and O placed
+    between sentinel bytes in one buffer, no byte outside O changes, and O is
+    the same as in a buffer of its own."""
+    w = W.small_variant(W.get("prefill"), N=300, B=2, Hq=3)
+    q, k, v = W.make_qkv(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    if layout == "NHD":
+        qd, kd, vd = _nhd(qd, kd, vd)
+    kw = dict(causal=w.causal, sm_scale=w.sm_scale, smooth_k=w.smooth_k, smooth_q=w.smooth_q, bq=w.bq, bk=w.bk,
+              pv_accum=pv_accum, tensor_layout=layout)
+    ref = sage.sage_attn_fwd(qd, kd, vd, **kw)
+    n = qd.numel()
+    guard = 4096  # elements on each side (16-byte aligned offsets keep O aligned)
+    buf = torch.full((n + 2 * guard,), -7.0, dtype=qd.dtype, device=qd.device)
+    out = buf[guard:guard + n].view(qd.shape)
+    sage.sage_attn_fwd(qd, kd, vd, out=out, **kw)
+    torch.cuda.synchronize()
+    assert sage.sage_last_device_error() == 0
+    sentinel = torch.full((guard,), -7.0, dtype=qd.dtype, device=qd.device)
+    assert torch.equal(buf[:guard].view(torch.int16), sentinel.view(torch.int16))
+    assert torch.equal(buf[guard + n:].view(torch.int16), sentinel.view(torch.int16))
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
