@@ -8,8 +8,10 @@
 //   psi_V:     per-channel FP8 E4M3, scale = amax / 448
 //   GEMV:      delta_S[i, j] = qbar_i . gamma(K_j)   (tcgen05 TF32, 3-term split)
 // Bit-exactness with the plain definitions: column sums are accumulated in
-// fp64 (the partial sums of bf16/fp16 inputs are exact, so the order does
-// not matter), divided in fp64 and rounded once to fp32; every division of
+// fp64 (the partial sums of bf16/fp16 inputs are exact -- 53 bits hold a sum
+// of up to 2^15 tokens whose magnitudes in one column lie within about 2^30
+// of each other, which attention inputs do -- so the order does not matter),
+// divided in fp64 and rounded once to fp32; every division of
 // the quantisers is an IEEE fp32 division (__fdiv_rn) -- per element it is
 // replaced by a multiplication with the reciprocal wherever that provably
 // gives the same code (quant8_i8 / quant_e4m3x2 below) -- and the INT8 rounding
@@ -126,18 +128,29 @@ __device__ __forceinline__ uint32_t quant_e2m1x8(const float (&x)[8], float s, f
   return cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
 }
 
-// CTA-wide max of non-negative floats; every thread gets the result.
-__device__ __forceinline__ float block_max_nonneg(float v, float* red) {
+// CTA-wide maxima of NB non-negative floats per thread, all in one pass (one
+// pair of CTA barriers for the NB values): out[nb] = max over the CTA of v[nb].
+// red holds NB x (warps) floats; out is visible to every thread on return.
+template <int NB>
+__device__ __forceinline__ void block_max_nonneg_n(float (&v)[NB], float* red, float* out) {
+  constexpr int NW = kThreads / 32;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[nb] = fmaxf(v[nb], __shfl_xor_sync(0xffffffffu, v[nb], o));
   const int w = threadIdx.x / 32;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[w] = v;
-  __syncthreads();
-  float r = 0.0f;
+  __syncthreads();  // red and out may still be read by an earlier reduction
+  if ((threadIdx.x & 31) == 0)
 #pragma unroll
-  for (int i = 0; i < kThreads / 32; ++i) r = fmaxf(r, red[i]);
-  return r;
+    for (int nb = 0; nb < NB; ++nb) red[nb * NW + w] = v[nb];
+  __syncthreads();
+  if (threadIdx.x < NB) {
+    float r = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) r = fmaxf(r, red[threadIdx.x * NW + i]);
+    out[threadIdx.x] = r;
+  }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -237,6 +250,7 @@ __device__ __forceinline__ void lds8(const T* p, float (&x)[8]) {
 }
 
 // INT8 codes of one 128-row tile in shared memory (rows past N are zero):
+// (s_red: NB x 8 floats)
 // per BQ-row block, scale = max |x - shift| / 127 over the valid rows, codes
 // rint(RN((x - shift) / scale)); writes the scales (s_k or s_q) and the codes
 // (k8 or q8).  SHIFT = false: the shift is zero and the block max runs on the
@@ -289,12 +303,7 @@ __device__ __forceinline__ void qk_encode(const T* sX, const float (*s_shift)[D]
         bm[nb] = __half2float(__ushort_as_half((unsigned short)m16));
     }
   }
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    const float m = block_max_nonneg(bm[nb], s_red);
-    if (threadIdx.x == 0) s_bmax[nb] = m;
-  }
-  __syncthreads();
+  block_max_nonneg_n<NB>(bm, s_red, s_bmax);
   float sc[NB], rc[NB];
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) {
@@ -379,7 +388,7 @@ __global__ void __launch_bounds__(kThreads) qk_quant_kernel(const __grid_constan
   extern __shared__ uint8_t qk_smem_raw[];
   T* sX = reinterpret_cast<T*>(align128(qk_smem_raw));
   __shared__ double s_sum[kThreads][8];
-  __shared__ float s_shift[NB][D], s_red[kThreads / 32], s_bmax[NB];
+  __shared__ float s_shift[NB][D], s_red[NB * (kThreads / 32)], s_bmax[NB];
   __shared__ uint64_t bar;
   const int bh = blockIdx.y, tile = blockIdx.x;
   const int64_t r0 = (int64_t)tile * kTile;
@@ -495,7 +504,8 @@ __global__ void __launch_bounds__(kThreads)
 // path reads K and V twice (statistics, then codes).  Here a CTA loads one
 // 128-token tile of K or V once, adds the tile's column sums (fp64) or
 // column max |V| into its head's totals (the atomics of the statistics pass:
-// fp64 sums of 16-bit inputs do not round, so the order does not matter),
+// fp64 sums of 16-bit inputs are exact in the range described at the top of
+// this file, so the order does not matter),
 // counts itself as published, and keeps the tile in shared memory until all
 // tiles of its (head, K|V) group have published; then it reads km or s_v
 // from the totals and writes its codes.
@@ -549,7 +559,7 @@ __global__ void __launch_bounds__(kThreads)
   T* sX = reinterpret_cast<T*>(sVt);
   __shared__ double s_pk[NW * D];                       // per-warp column sums (K group)
   unsigned* s_pv = reinterpret_cast<unsigned*>(s_pk);  // per-warp column max |V| bits (V group)
-  __shared__ float s_shift[NB][D], s_red[NW], s_bmax[NB];
+  __shared__ float s_shift[NB][D], s_red[NB * NW], s_bmax[NB];
   __shared__ uint64_t bar;
   __shared__ int s_item, s_ok;
   const int tiles = (int)(a.Np / kTile);
