@@ -31,7 +31,7 @@ def gpu_quant(w: W.Workload, q, k, v, pv_accum: int = sage.PV_TWO_LEVEL):
 
 def gpu_attention(w: W.Workload, q, k, v, pv_accum: int = sage.PV_TWO_LEVEL):
     p, ws, view, (qd, kd, vd) = gpu_quant(w, q, k, v, pv_accum)
-    o = torch.empty_like(qd)
+    o = torch.full_like(qd, float("nan"))  # a row the kernel does not write stays NaN
     sage.sage_attn_fwd_quantized(view, o, p)
     torch.cuda.synchronize()
     assert sage.sage_last_device_error() == 0
@@ -126,7 +126,7 @@ def gpu_quant_nvfp4(w: W.Workload, q, k, v):
 
 def gpu_attention_nvfp4(w: W.Workload, q, k, v):
     p, ws, view, (qd, kd, vd) = gpu_quant_nvfp4(w, q, k, v)
-    o = torch.empty_like(qd)
+    o = torch.full_like(qd, float("nan"))  # a row the kernel does not write stays NaN
     sage.sage_attn_fwd_nvfp4_quantized(view, o, p)
     torch.cuda.synchronize()
     assert sage.sage_last_device_error() == 0
