@@ -20,9 +20,11 @@
 // K / V tile.  512 threads in four warpgroups:
 //   WG0  warp 0: TMA producer (Q tiles once, K_j / V_j^T through a ring)
 //        warp 1: MMA issuer (one thread) and TMEM owner; warps 2-3 idle
-//   WG1  softmax of Q tile 0    (thread = one Q row = one TMEM lane)
-//   WG2  softmax of Q tile 1
-//   WG3  level-2 accumulation O = alpha O + O_t for both tiles, and the epilogue
+//   WG1  softmax of Q tile 0    (thread = one Q row = one TMEM lane); in two-level
+//        mode also the level-2 sum O = alpha O + O_t of its tile
+//   WG2  the same for Q tile 1
+//   WG3  (TMEM accumulator mode) the rescale of O before each P V; the epilogue
+//        of both tiles (output through TMA bulk stores)
 // The two softmax warpgroups run concurrently (two softmax warps per SM
 // sub-partition hide each other's latencies).  TMEM (512 columns): S_i at
 // [128 i, 128 i + 128), holding the magic fill 0x4B400000 between uses (QK^T
@@ -31,8 +33,8 @@
 // j + 1 never waits for P V(j).
 // Two P~V accumulation modes (template TWO_LEVEL):
 //   two-level: PV(i, j) writes a fresh O_t into S_i's columns (S is dead once
-//     the softmax read it); the correction warpgroup adds it into O_i on CUDA
-//     cores: O_i = alpha O_i + O_t (SageAttention2 Algorithm 1, level 2).
+//     the softmax read it); the softmax warpgroup of tile i adds it into O_i on
+//     CUDA cores: O_i = alpha O_i + O_t (SageAttention2 Algorithm 1, level 2).
 //   TMEM accumulator: PV(i, j) accumulates into O_i itself (tcgen05 keeps the
 //     FP8 products' sum in full FP32); before it, the correction warpgroup
 //     rescales the rows of O_i whose max grew (alpha != 1; alpha == 1 is exact).
@@ -116,8 +118,8 @@ struct Bars {
   uint64_t* p_empty;   // [tile][buffer]  the P V that read that P buffer retired (tcgen05.commit)
   uint64_t* ot_full;   // [2]  P V of tile i retired              (tcgen05.commit)
   uint64_t* r_free;    // [2]  S_i columns hold the magic fill again and may take the next QK^T
-                       //      (TMEM accumulator: the softmax refilled them; two-level: the
-                       //      correction consumed O_t_i and refilled them); one arrival per warp
+                       //      (the softmax refilled them; in two-level mode after it read
+                       //      O_t_i there); one arrival per warp
   uint64_t* l_ready;   // [2]  final l of tile i in shared memory (128 threads)
   uint64_t* o_ready;   // [2]  (TMEM accumulator mode) O_i rescaled for the next P V (one per warp)
   uint64_t* mma_done;  // all tensor-core work of the CTA retired (one commit at the end)
