@@ -11,8 +11,8 @@ import oracle
 from quantized_attention_block_b200 import sage
 from quantized_attention_block_b200 import workloads as W
 
-from harness import (compare_out, compare_quant_nvfp4, gpu_attention_nvfp4, gpu_nvfp4_in_oracle_layout,
-                     gpu_quant_nvfp4, oracle_quant_nvfp4, oracle_rows_nvfp4)
+from harness import (accept_boundary_rows, compare_out, compare_quant_nvfp4, gpu_attention_nvfp4,
+                     gpu_nvfp4_in_oracle_layout, gpu_quant_nvfp4, oracle_quant_nvfp4, oracle_rows_nvfp4)
 
 pytestmark = pytest.mark.gpu
 
@@ -162,3 +162,53 @@ def test_nvfp4_full_size_quant_bit_exact_and_sampled_attention():
     for (b, h, r0, r1), ref in zip(jobs, refs):
         m, ok = compare_out(ref, out[b, h, r0:r1])
         assert ok, ((b, h, r0, r1), m)
+
+
+def _random_case(i: int):
+    """A seeded random NVFP4 configuration (d = 128): sequence length, batch,
+    GQA ratio, causal mask, smooth K / smooth Q, smooth-Q block size, dtype."""
+    rng = np.random.default_rng(2000 + i)
+    hkv = int(rng.choice([1, 2]))
+    g = int(rng.choice([1, 2, 4]))
+    smooth_q = bool(rng.random() < 0.5)
+    w = NV.with_(
+        name=f"nvfp4_rand{i}",
+        B=int(rng.choice([1, 2])),
+        Hq=hkv * g,
+        Hkv=hkv,
+        N=int(rng.choice([1, 2, 63, 64, 65, 127, 128, 129]) if rng.random() < 0.3 else rng.integers(2, 700)),
+        dtype=torch.float16 if rng.random() < 0.3 else torch.bfloat16,
+        causal=bool(rng.random() < 0.5),
+        smooth_k=bool(rng.random() < 0.8),
+        smooth_q=smooth_q,
+        bq=int(rng.choice([64, 128])),
+        seed=int(rng.integers(0, 2**31 - 1)),
+    )
+    if g > 1:
+        # (a bias shared by Q and K needs as many K heads as Q heads)
+        w = w.with_(qk_shared_bias_std=0.0, k_bias_std=3.0)
+    return w
+
+
+@pytest.mark.parametrize("i", range(32))
+def test_nvfp4_random_configuration_matches_oracle(i):
+    """Codes and scales bit-exact and every output row element by element on
+    seeded random configurations (the output starts as NaN).  A row whose FP4
+    code of P sits on a rounding boundary may be matched against the oracle
+    with the score scale moved within the kernel's fp32 error
+    (harness.accept_boundary_rows, at most 1% of the rows)."""
+    w = _random_case(i)
+    q, k, v = W.make_qkv(w)
+    p, ws, view, o = gpu_attention_nvfp4(w, q, k, v)
+    quant = oracle_quant_nvfp4(w, q, k, v)
+    bad = compare_quant_nvfp4(w, gpu_nvfp4_in_oracle_layout(view, p, ws), quant)
+    assert not bad, (w, bad)
+    out = o.float().cpu().numpy()
+    refs = np.stack([np.stack([oracle_rows_nvfp4(w, quant, b, h, 0, w.N) for h in range(w.Hq)])
+                     for b in range(w.B)])
+    refs, accepted, failing = accept_boundary_rows(
+        w, out, refs, lambda b, h, r, sm: oracle.attention_nvfp4_head(quant, b, h, r, r + 1, bq=w.bq,
+                                                                        causal=w.causal, sm_scale=sm)[0])
+    assert not failing, (w, failing)
+    m, ok = compare_out(refs, out)
+    assert ok, (w, m, accepted)

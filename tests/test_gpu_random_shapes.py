@@ -3,7 +3,10 @@ hand-picked edge cases: sequence length (ragged or not, down to 1), batch, GQA
 ratio, head dim, causal mask, smooth K / smooth Q, Q and K block sizes, input
 dtype and PV accumulation mode all drawn at random.  Each case checks the
 quantised tensors bit-exactly and every output row element by element against
-the oracle (the output starts as NaN, so an unwritten row fails)."""
+the oracle (the output starts as NaN, so an unwritten row fails); a row whose
+E4M3 code of P sits on a rounding boundary may be matched with the score scale
+moved within the kernel's fp32 error (harness.accept_boundary_rows, at most 1%
+of the rows)."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +14,8 @@ import torch
 from quantized_attention_block_b200 import sage
 from quantized_attention_block_b200 import workloads as W
 
-from harness import compare_out, compare_quant, gpu_attention, oracle_quant, oracle_rows
+import oracle
+from harness import accept_boundary_rows, compare_out, compare_quant, gpu_attention, oracle_quant, oracle_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -59,5 +63,9 @@ def test_random_configuration_matches_oracle(i):
     assert not bad, (w, bad)
     out = o.float().cpu().numpy()
     refs = np.stack([np.stack([oracle_rows(w, quant, b, h, 0, w.N) for h in range(w.Hq)]) for b in range(w.B)])
+    refs, accepted, failing = accept_boundary_rows(
+        w, out, refs, lambda b, h, r, sm: oracle.attention_sage_head(quant, b, h, r, r + 1, bq=w.bq, bk=w.bk,
+                                                                       causal=w.causal, sm_scale=sm)[0])
+    assert not failing, (w, mode, failing)
     m, ok = compare_out(refs, out)
-    assert ok, (w, mode, m)
+    assert ok, (w, mode, m, accepted)
