@@ -39,9 +39,9 @@ FP4_PER_BF16 = 4.0  # nominal dense ratio 9 / 2.25 PFLOP/s
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch of the prefill workload: one ncu capture of attn_i8f8_kernel at B=3
-# (431.3 + 73.3 MB), scaled to B=4 by the number of heads.  Valid only for the
+# (431.9 + 69.2 MB), scaled to B=4 by the number of heads.  Valid only for the
 # kernel sources it was taken on (hash below); any other source reports null.
-ATTN_TRAFFIC = {"bytes": (431317504 + 73300992) * 4 / 3, "src_sha256_16": "1f2e753dfb95abda",
+ATTN_TRAFFIC = {"bytes": (431864064 + 69236480) * 4 / 3, "src_sha256_16": "d608e0ce163c0c7c",
                 "workload": "llm_prefill_causal_B4_H32_N4096_d128"}
 
 

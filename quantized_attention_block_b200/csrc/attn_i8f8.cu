@@ -67,9 +67,18 @@ constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 #endif
 constexpr unsigned kPolyPairs = SAGE_POLY_PAIRS;
 
-// per-warpgroup register budgets after setmaxnreg (sum x 128 <= 65536)
-constexpr uint32_t kRegsProducer = 40, kRegsSoftmax = 192, kRegsCorrection = 88;
-static_assert(kRegsProducer + 2 * kRegsSoftmax + kRegsCorrection <= 512, "register split exceeds the launch");
+// per-warpgroup register budgets after setmaxnreg (sum x 128 <= 65536).  In
+// TMEM-accumulator mode 56 / 192 / 72 (with the correction's rescale loop not
+// unrolled) leaves no warpgroup spilling; the two-level instances keep
+// 40 / 192 / 88, which measured faster for them than any spill-free split.
+template <bool TWO_LEVEL>
+constexpr uint32_t kRegsProducer = TWO_LEVEL ? 40 : 56;
+constexpr uint32_t kRegsSoftmax = 192;
+template <bool TWO_LEVEL>
+constexpr uint32_t kRegsCorrection = TWO_LEVEL ? 88 : 72;
+static_assert(kRegsProducer<true> + 2 * kRegsSoftmax + kRegsCorrection<true> <= 512 &&
+                  kRegsProducer<false> + 2 * kRegsSoftmax + kRegsCorrection<false> <= 512,
+              "register split exceeds the launch");
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -281,7 +290,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   tc_fence_after();
 
   if (wg == 0) {
-    regs_dec<kRegsProducer>();
+    regs_dec<kRegsProducer<TWO_LEVEL>>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
       // (Q and K / V tiles 0 .. kStages - 1 went out before the first barrier)
@@ -583,7 +592,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     mbar_arrive(&bar.l_ready[ti]);
   } else {
     // ------------------------------------------------------------ correction + epilogue
-    regs_dec<kRegsCorrection>();
+    regs_dec<kRegsCorrection<TWO_LEVEL>>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -614,7 +623,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           const float alpha = s_alpha[(i * 2 + (j & 1)) * 128 + row];
           if (__any_sync(0xffffffffu, alpha != 1.0f)) {
             const uint32_t tO = tmem + 256 + D * i + lane_off;
-#pragma unroll
+            // (not unrolled: it keeps this warpgroup within its 72 registers)
+#pragma unroll 1
             for (int c = 0; c < D; c += 32) {
               tmem_ld32(tO + c, x);
               tmem_ld_wait();
