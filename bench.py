@@ -331,9 +331,25 @@ def run_sage(w: W.Workload, steps: int, warmup: int, ws: int, rank: int, local: 
         torch.cuda.synchronize()
         assert sage.sage_last_device_error() == 0
         ms_e2e = _max_over_ranks(t0.elapsed_time(t1) / e_steps, ws)
-        res["e2e"] = {"ms_step": ms_e2e, "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+        # The same host->device copies alone (the step's input bytes over the
+        # link, nothing else): the time the pipelined step cannot go below.
+        qb, kb, vb, _ = bufs[0]
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        c0.record(s_in)
+        with torch.cuda.stream(s_in):
+            for _ in range(e_steps):
+                qb.copy_(qh, non_blocking=True)
+                kb.copy_(kh, non_blocking=True)
+                vb.copy_(vh, non_blocking=True)
+        c1.record(s_in)
+        torch.cuda.synchronize()
+        ms_h2d = _max_over_ranks(c0.elapsed_time(c1) / e_steps, ws)
+        h2d_bytes = 3 * q.numel() * q.element_size()
+        res["e2e"] = {"ms_step": ms_e2e, "h2d_bytes_per_step": h2d_bytes,
                       "d2h_bytes_per_step": o.numel() * o.element_size(), "steps": e_steps,
-                      "pipelined": "double-buffered: copies of step i overlap the attention of step i-1"}
+                      "pipelined": "double-buffered: copies of step i overlap the attention of step i-1",
+                      "h2d_copy_ms": ms_h2d, "h2d_gbs": h2d_bytes / (ms_h2d * 1e-3) / 1e9}
         del bufs, ohs
     del wsp, qd, kd, vd, o
     torch.cuda.empty_cache()
@@ -531,7 +547,10 @@ def main():
         e = res["e2e"]
         line["e2e"] = {"value": weak_scaling_tops(ops, e["ms_step"], ws), "unit": "TOPS",
                        "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
-                       "ms_step": e["ms_step"], "pipelined": e["pipelined"]}
+                       "ms_step": e["ms_step"], "pipelined": e["pipelined"],
+                       # the input copies alone over the host link: the bound of the pipelined step
+                       "h2d_copy_ms_per_step": e["h2d_copy_ms"], "h2d_gbs": e["h2d_gbs"],
+                       "copy_bound_frac": e["h2d_copy_ms"] / e["ms_step"]}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         # about 10-15 s on a 16-core host: three batches' worth of heads, the 32
         # longest Q tiles of each
